@@ -1,0 +1,188 @@
+/*
+ * da2.h -- C ABI of the DraftAttention2 attention hot path for NVIDIA B200
+ * (sm_100a).  Method: "DraftAttention2" (paperpeel.com/paper/2609.32628.md).
+ *
+ * The three calls follow the paper's statement of the problem (Sec. 3.1,
+ * 3.3; App. C.1-C.2): per-head Q, K, V; a region partition of every frame;
+ * operand preparation; draft-guided routing under precision budgets; one
+ * block-sparse mixed-precision attention:
+ *
+ *   da2_prepare   -- fused gather + pooling + FP8/NVFP4 quantization (Sec. 3.3
+ *                    "Fused quantization and reordering", Fig. 3b)
+ *   da2_plan      -- draft map, per-head ranking, quotas, precision
+ *                    assignment, per-row block lists (Eq. 3; Sec. 3.1 "Joint
+ *                    allocation of sparsity and precision"; App. C.1)
+ *   da2_attention -- phased FP8 / NVFP4 block-sparse attention with one
+ *                    softmax state and one output accumulator, original token
+ *                    order restored on store (Sec. 3.3 "Phased execution",
+ *                    "Cross-precision accumulation"; App. B.3, C.1)
+ *
+ * Conventions for every call
+ *   - Pointers marked (device) are CUDA device pointers, owned by the caller;
+ *     the library never allocates on the call path.  The handle owns only
+ *     its partition tables (allocated by da2_create, freed by da2_destroy).
+ *   - All device work is asynchronous on the given stream; the call returns
+ *     after enqueueing.  A stream of 0 means the legacy default stream.
+ *   - Return value: DA2_OK or a negative DA2_ERR_* code; nothing is enqueued
+ *     when an argument check fails.  DA2_ERR_CUDA means a launch failed; the
+ *     CUDA error string is available from da2_last_cuda_error().
+ *   - Device-side waits inside the kernels are bounded; when one gives up the
+ *     kernel records it and returns; da2_check_device_status() reports it as
+ *     DA2_ERR_TIMEOUT (it synchronizes the stream it is given).
+ *   - Inputs are bf16, finite.  NaN / Inf inputs give undefined results.
+ *
+ * Geometry.  The sequence holds F frames of Hv x Wv tokens in raster order
+ * (token t = f*Hv*Wv + y*Wv + x).  Each frame is split into
+ * R_f = ceil(Hv*Wv/64) connected regions of balanced size (App. C.2); region
+ * j of frame f is block a = f*R_f + j, R = F*R_f blocks, Npad = 64*R packed
+ * slots.  Slots >= n_a of block a are padding.
+ */
+#ifndef DA2_H
+#define DA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DA2_OK 0
+#define DA2_ERR_ARG -1     /* null pointer, bad shape, bad stride, budget > 100 %, C != 64, d not 64/128 */
+#define DA2_ERR_ARCH -2    /* current device is not sm_100 */
+#define DA2_ERR_CUDA -3    /* a CUDA call or launch failed */
+#define DA2_ERR_TIMEOUT -4 /* a bounded device-side wait gave up */
+
+typedef struct {
+    int B, H;      /* batch, heads */
+    int d;         /* head dim: 64 or 128 */
+    int F, Hv, Wv; /* frames and latent frame size; N = F*Hv*Wv tokens */
+    int C;         /* region capacity = attention block size; must be 64 */
+} da2_shape;
+
+typedef struct {
+    int bp_fp8;    /* basis points of the R^2 region pairs of each head kept in FP8 */
+    int bp_fp4;    /* basis points kept in NVFP4; bp_fp8 + bp_fp4 <= 10000; the rest is skipped */
+    double lambda; /* max-pool branch weight of the draft map (Eq. 3); 0 = average only */
+} da2_budget;
+
+typedef struct da2_ctx* da2_handle;
+
+/* Byte sizes of every caller-owned buffer for a shape (filled by da2_sizes). */
+typedef struct {
+    int R, Rf, Npad;
+    /* prepared operands */
+    size_t desc, q8, k8, v8, q4, k4, v4, sfq, sfk, sfv, scale, vmax;
+    /* plan outputs and scratch */
+    size_t prec, cnt, kidx, A, plan_scratch;
+} da2_sizes_t;
+
+/* Prepared operands (da2_prepare output, da2_attention input).  All device.
+ *   desc  f64 [4][B][H][R][d]   Qbar, Qmax, Kbar, Kmax (Eq. 2): mean over the
+ *                               n_a valid slots (fp64 sum in slot order, then
+ *                               one fp64 divide) and channel-wise max.
+ *   q8,k8 u8 [B][H][R][64*d]    e4m3 codes of the 64 x d tile, tcgen05 K-major
+ *                               no-swizzle layout: byte (row r, col c) at
+ *                               ((r/8)*(d/16) + c/16)*128 + (r%8)*16 + c%16.
+ *   v8    u8 [B][H][R][d*64]    e4m3 codes of V^T (d rows x 64 slots), same
+ *                               layout with 64 columns.
+ *   q4,k4 u8 [B][H][R][64*d/2]  e2m1 codes, two per byte (even column in the low
+ *                               nibble), same layout over d/2 byte columns.
+ *   v4    u8 [B][H][R][d*32]    e2m1 codes of V^T, same layout, 32 byte columns.
+ *   sfq   u8 [B][H][R][64][d/16] ue4m3 scale of each 16-channel group of Q.
+ *   sfk   u8 [B][H][R][512]     ue4m3 scales of K (16-channel groups) in the
+ *                               tensor-memory copy atom: byte 16*(n%32) +
+ *                               4*(2*(c/64) + n/32) + (c%64)/16 for key slot n,
+ *                               channel c (bytes not covered are zero).
+ *   sfv   u8 [B][H][R][512]     ue4m3 scales of V^T (16-slot groups): byte
+ *                               16*(c%32) + 4*(c/32) + j/16 for channel c, slot j.
+ *   scale f32 [6][B][H][R]      FP8 tile scales of Q, K, V (amax/448), then
+ *                               NVFP4 tile scales of Q, K, V (amax/2688).
+ *   vmax  f32 [2][B][H]         per head max of the FP8 and of the NVFP4 V tile
+ *                               scales (the phase units are vmax/448, vmax/2688).
+ */
+typedef struct {
+    double* desc;
+    uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
+    float* scale;
+    float* vmax;
+} da2_prepared;
+
+/* Plan (da2_plan output, da2_attention input).  All device.
+ *   prec    u8  [B][H][R][R]  precision of pair (a,b): 8, 4 or 0 (skip)
+ *   cnt     i32 [2][B][H][R]  per query block: number of FP8, of NVFP4 key blocks
+ *   kidx    u16 [B][H][R][R]  row a: its FP8 key blocks ascending, then its
+ *                             NVFP4 key blocks ascending (cnt entries used)
+ *   A       f64 [B][H][R][R]  the draft map (Eq. 3), left readable after the call
+ *   scratch                   plan_scratch bytes of working memory
+ */
+typedef struct {
+    uint8_t* prec;
+    int32_t* cnt;
+    uint16_t* kidx;
+    double* A;
+    void* scratch;
+} da2_plan_bufs;
+
+/* Validate the shape, build the region partition on the host (App. C.2
+ * reading: balanced R_f regions, boustrophedon band walk, smallest total
+ * perimeter among connected candidates) and copy the slot tables to the
+ * current device.  *out receives the handle.  Errors: DA2_ERR_ARG,
+ * DA2_ERR_ARCH, DA2_ERR_CUDA. */
+int da2_create(const da2_shape* shape, da2_handle* out);
+
+/* Host-only: the partition of a shape without a device.  Fills
+ * slot_token[64*R] (token of each packed slot, -1 = padding) and n_a[R]
+ * (valid tokens per block), R = F*ceil(Hv*Wv/64), and returns R; returns
+ * DA2_ERR_ARG for a non-positive size.  Either pointer may be NULL. */
+int da2_partition(int F, int Hv, int Wv, int32_t* slot_token, int32_t* n_a);
+
+/* Free the handle and its device tables.  NULL is accepted. */
+int da2_destroy(da2_handle h);
+
+/* Sizes of every caller-owned buffer for the handle's shape. */
+int da2_sizes(da2_handle h, da2_sizes_t* out);
+
+/* Host copies of the partition tables: slot_token[Npad] (token of each packed
+ * slot, -1 for padding) and n_a[R] (valid tokens per block).  Either may be
+ * NULL. */
+int da2_tables(da2_handle h, int32_t* slot_token, int32_t* n_a);
+
+/* Fused operand preparation (Sec. 3.3, Fig. 3b).  q, k, v: bf16 (device),
+ * element (b,h,t,c) at p[b*s[0] + h*s[1] + t*s[2] + c] with strides s[] in
+ * elements (s[3] must be 1; the base and s[2] must keep rows 16-byte aligned).
+ * Gathers every 64-slot block through the partition, writes the pooled
+ * descriptors and the FP8 / NVFP4 operands and scales into *out. */
+int da2_prepare(da2_handle h, const void* q, const void* k, const void* v, const int64_t strides[4],
+                const da2_prepared* out, void* stream);
+
+/* Draft-guided routing (Eq. 3; Sec. 3.1; App. C.1): A in fp64 with a fixed
+ * operation order, per-head ranking of all R^2 pairs by A (ties to the
+ * smaller pair index a*R+b), quotas T8 = floor(R^2 bp_fp8/10^4),
+ * Tkeep = floor(R^2 (bp_fp8+bp_fp4)/10^4); ranks below T8 -> FP8, below
+ * Tkeep -> NVFP4, the rest skipped; per-row lists.  Errors: DA2_ERR_ARG for
+ * a budget outside [0, 10000] or lambda outside [0, 1]. */
+int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, const da2_plan_bufs* plan,
+             void* stream);
+
+/* Block-sparse mixed-precision attention (Sec. 3.3; App. B.3, C.1).  out:
+ * bf16 (device), [B][H][N][d] with strides out_strides[] in elements
+ * (out_strides[3] == 1); every token row is written (rows with no retained
+ * valid key get zeros). */
+int da2_attention(da2_handle h, const da2_prepared* prep, const da2_plan_bufs* plan, void* out,
+                  const int64_t out_strides[4], void* stream);
+
+/* Synchronize `stream` and report whether a bounded device wait gave up
+ * since the last call (DA2_ERR_TIMEOUT), clearing the flag. */
+int da2_check_device_status(da2_handle h, void* stream);
+
+/* Static description of a status code. */
+const char* da2_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* da2_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DA2_H */

@@ -579,7 +579,9 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                      const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
                      const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
                      const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
-                     const float* vmax, const int* cnt, const uint16_t* kidx, int flags, double* out) {
+                     const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
+                     double* out) {
+    /* sel: NULL, or one byte per (b,h,block); blocks with sel == 0 are not computed. */
     o_geom g;
     int qops = flags & 1, qw = flags & 2, units = flags & 4;
     if (qw && !units) return -2;
@@ -601,6 +603,7 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
         float sig8 = vmax[bh] / 448.0f, sig4 = vmax[BH + bh] / 2688.0f;
         for (int a = 0; a < R; ++a) {
             size_t ba = (size_t)bh * R + a;
+            if (sel && !sel[ba]) continue;
             int n8 = cnt[ba], n4 = cnt[BHR + ba], nq = g.n_a[a];
             const uint16_t* L = kidx + ba * R;
             gather_tile(&g, q, bh, a, Qt);

@@ -56,7 +56,7 @@ def lib():
         L.oracle_prepare.argtypes = [i] * 6 + [P] * 3 + [P] * 13
         L.oracle_draft.argtypes = [i, i, i, P, ctypes.c_double, P]
         L.oracle_assign.argtypes = [i, i, P, i, i, P, P, P]
-        L.oracle_attention.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P]
+        L.oracle_attention.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P, P]
         L.oracle_dense.argtypes = [i, i, i, P, P, P, P]
         L.oracle_num_threads.restype = i
         _lib = L
@@ -195,15 +195,20 @@ def assign(A: np.ndarray, bp8: int, bp4: int) -> Plan:
     return plan
 
 
-def attention(q, k, v, F, Hv, Wv, prep: Prepared, plan: Plan, flags: int = 7) -> np.ndarray:
-    """Block-sparse mixed-precision attention, f64 [B,H,N,d] in token order."""
+def attention(q, k, v, F, Hv, Wv, prep: Prepared, plan: Plan, flags: int = 7, blocks=None) -> np.ndarray:
+    """Block-sparse mixed-precision attention, f64 [B,H,N,d] in token order.
+
+    blocks: optional boolean [B,H,R] selecting the query blocks to compute
+    (the other tokens stay 0)."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, H, N, d = qb.shape
     out = np.zeros((B, H, N, d), np.float64)
+    sel = None if blocks is None else np.ascontiguousarray(blocks, np.uint8)
     rc = lib().oracle_attention(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(vb), _p(prep.q8), _p(prep.k8),
                                 _p(prep.v8t), _p(prep.s8), _p(prep.q4), _p(prep.k4), _p(prep.v4t),
                                 _p(prep.sfq), _p(prep.sfk), _p(prep.sfv), _p(prep.g4), _p(prep.vmax),
-                                _p(plan.cnt), _p(plan.kidx), int(flags), _p(out))
+                                _p(plan.cnt), _p(plan.kidx), int(flags),
+                                None if sel is None else _p(sel), _p(out))
     if rc:
         raise ValueError(f"oracle_attention failed ({rc})")
     return out

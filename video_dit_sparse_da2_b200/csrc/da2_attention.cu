@@ -1,0 +1,537 @@
+// da2_attention.cu -- phased block-sparse mixed-precision attention for
+// sm_100a ("DraftAttention2", Sec. 3.3 "Phased execution" Eq. 7 and
+// "Cross-precision accumulation" Eq. 8; App. B.3 shared normalization;
+// App. C.1 formats and empty rows).
+//
+// Work item = two query blocks (a0 = 2i, a1 = 2i+1) of one head stacked into
+// one M = 128 tile: the block-scaled NVFP4 MMA has M = 128 per CTA, the
+// method's query blocks have 64 tokens.  The kernel walks the union of the
+// two blocks' key lists, first all 8-bit key blocks (ascending), then all
+// 4-bit key blocks (ascending); a row takes part in a step only when its own
+// block kept that key block at that precision, so every row sees exactly its
+// own list in the order of the method.
+//
+// Roles (192 threads, persistent CTAs, one per SM):
+//   warps 0-3  softmax: thread r owns row r of the tile.  Reads S from tensor
+//              memory, keeps the row max m and the unquantized denominator l
+//              (App. B.3), quantizes the weights (FP8: e4m3 of p times the
+//              value-tile scale over the phase unit; NVFP4: the same product
+//              quantized per 16 keys with an e4m3 scale) into shared memory,
+//              rescales its row of O when m grows and once at the phase
+//              switch (sigma8 -> sigma4, the change of units of Eq. 8), and
+//              in the epilogue divides by l, converts to bf16 and stores the
+//              row at its original token position.
+//   warp 4     MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
+//              kind::mxf4nvf4 block16) into one of two S buffers in tensor
+//              memory, then O += P V into the single O accumulator.
+//   warp 5     loader (one thread): bulk async copies of the K / V tiles
+//              (pre-tiled by the preparation kernel) into a 3-stage ring.
+// Every mbarrier wait is bounded; a stuck wait sets the status word, all
+// roles drain their own outstanding work and the CTA frees tensor memory
+// before returning.
+#include "da2_common.cuh"
+#include "da2_kernels.h"
+
+namespace da2 {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+// tensor-memory column map
+constexpr uint32_t kColO = 0;       // O accumulator, D columns
+constexpr uint32_t kColS = 128;     // two S buffers of 64 columns
+constexpr uint32_t kColSfq = 256;   // Q scale factors, 4 columns per 64-channel chunk
+constexpr uint32_t kColSfk = 264;   // K scale factors, 2 buffers x 4 columns
+constexpr uint32_t kColSfp = 272;   // P scale factors, 2 buffers x 4 columns
+constexpr uint32_t kColSfv = 280;   // V scale factors, 2 buffers x 4 columns
+
+struct Entry {  // one step of the merged list
+    static __device__ __forceinline__ uint32_t make(int kb, int phase, int mask) {
+        return (uint32_t)kb | ((uint32_t)phase << 16) | ((uint32_t)mask << 17);
+    }
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t kmajor_off(int row, int chunk, int row_bytes) {
+    return ((row >> 3) * (row_bytes >> 4) + chunk) * 128 + (row & 7) * 16;
+}
+
+template <int D>
+struct Smem {
+    // byte offsets inside the dynamic shared memory block
+    static constexpr uint32_t q8 = 0;                          // 128 x D
+    static constexpr uint32_t q4 = q8 + 128 * D;               // 128 x D/2
+    static constexpr uint32_t sfq = q4 + 64 * D;               // D/64 atoms of 512
+    static constexpr uint32_t stage = sfq + 1024;              // kStages x stage_bytes
+    static constexpr uint32_t k_off = 0, v_off = 64 * D, ksf_off = 128 * D, vsf_off = 128 * D + 512;
+    static constexpr uint32_t stage_bytes = 128 * D + 1024;
+    static constexpr uint32_t p = stage + kStages * stage_bytes;  // 2 x (128 x 64 + 512)
+    static constexpr uint32_t p_bytes = 128 * 64 + 512;
+    static constexpr uint32_t bitmap = p + 2 * p_bytes;        // 4 x 128 words
+    static constexpr uint32_t list = bitmap + 4 * 128 * 4;     // entries
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
+    using L = Smem<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s[2], bar_p[2], bar_pv[2],
+        bar_drain;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ int n_ent_sh[2];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int R = p.R, BH = p.B * p.H;
+    const int pairs = (R + 1) / 2;
+    const int items = BH * pairs;
+    const int nwords = (R + 31) / 32;
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + L::bitmap);
+    uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::list);
+    volatile int* abort_v = &abort_sh;
+
+    if (tid == 0) {
+        mbar_init(&bar_q, 1);
+        mbar_init(&bar_sfq, kSoftmaxThreads);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bar_full[s], 1);
+            mbar_init(&bar_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar_s[s], 1);
+            mbar_init(&bar_p[s], kSoftmaxThreads);
+            mbar_init(&bar_pv[s], 1);
+        }
+        mbar_init(&bar_drain, 1);
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base_sh, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    uint32_t gstep = 0;  // entries processed by this CTA before the current item
+    uint32_t nitem = 0;  // items processed by this CTA
+    uint32_t loads_issued = 0;  // loader: stage fills issued (for the final drain)
+    bool mma_issued = false;
+
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++nitem) {
+        __syncthreads();
+        if (*abort_v) break;
+        const int bh = item / pairs, pr = item % pairs;
+        const int a0 = 2 * pr, a1 = 2 * pr + 1;
+        const bool has1 = a1 < R;
+
+        // ---- merged step list: union of the two rows' lists per phase
+        for (int i = tid; i < 4 * nwords; i += kThreads) bitmap[i] = 0u;
+        __syncthreads();
+        for (int hf = 0; hf < (has1 ? 2 : 1); ++hf) {
+            const size_t row = (size_t)bh * R + (hf ? a1 : a0);
+            const int n8 = p.cnt[row], n4 = p.cnt[(size_t)BH * R + row];
+            const uint16_t* L0 = p.kidx + row * R;
+            for (int i = tid; i < n8 + n4; i += kThreads) {
+                const int kb = L0[i];
+                if (kb >= R) { atomicOr(p.status, DA2_DEV_BADINDEX); continue; }
+                const int ph = i < n8 ? 0 : 1;
+                atomicOr(&bitmap[(ph * 2 + hf) * nwords + (kb >> 5)], 1u << (kb & 31));
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int base = 0;
+            for (int ph = 0; ph < 2; ++ph) {
+                for (int w0 = 0; w0 < nwords; w0 += 32) {
+                    const int w = w0 + lane;
+                    const uint32_t m0 = w < nwords ? bitmap[(ph * 2 + 0) * nwords + w] : 0u;
+                    const uint32_t m1 = w < nwords ? bitmap[(ph * 2 + 1) * nwords + w] : 0u;
+                    uint32_t u = m0 | m1;
+                    const int c = __popc(u);
+                    int incl = c;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    int pos = base + incl - c;
+                    while (u) {
+                        const int bit = __ffs(u) - 1;
+                        u &= u - 1;
+                        const int mask = ((m0 >> bit) & 1) | (((m1 >> bit) & 1) << 1);
+                        list[pos++] = Entry::make(w * 32 + bit, ph, mask);
+                    }
+                    base += __shfl_sync(0xffffffffu, incl, 31);
+                }
+                if (lane == 0) n_ent_sh[ph] = base - (ph ? n_ent_sh[0] : 0);
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        const int n8e = n_ent_sh[0], n_ent = n_ent_sh[0] + n_ent_sh[1];
+
+        if (warp == 5) {
+            // ================================================== loader
+            if (lane == 0) {
+                const size_t t0 = (size_t)bh * R + a0;
+                const uint32_t qb8 = 64 * D, qb4 = 32 * D;
+                mbar_expect_tx(&bar_q, (has1 ? 2u : 1u) * (qb8 + qb4));
+                bulk_g2s(smem + L::q8, p.q8 + t0 * qb8, qb8, &bar_q);
+                bulk_g2s(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
+                if (has1) {
+                    bulk_g2s(smem + L::q8 + qb8, p.q8 + (t0 + 1) * qb8, qb8, &bar_q);
+                    bulk_g2s(smem + L::q4 + qb4, p.q4 + (t0 + 1) * qb4, qb4, &bar_q);
+                }
+                for (int j = 0; j < n_ent; ++j) {
+                    const uint32_t g = gstep + j, st = g % kStages;
+                    if (!mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status)) break;
+                    const uint32_t e = list[j];
+                    const int kb = e & 0xFFFF, ph = (e >> 16) & 1;
+                    const size_t tk = (size_t)bh * R + kb;
+                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                    if (ph == 0) {
+                        mbar_expect_tx(&bar_full[st], 2 * 64 * D);
+                        bulk_g2s(sb + L::k_off, p.k8 + tk * (64 * D), 64 * D, &bar_full[st]);
+                        bulk_g2s(sb + L::v_off, p.v8 + tk * (64 * D), 64 * D, &bar_full[st]);
+                    } else {
+                        mbar_expect_tx(&bar_full[st], 2 * 32 * D + 1024);
+                        bulk_g2s(sb + L::k_off, p.k4 + tk * (32 * D), 32 * D, &bar_full[st]);
+                        bulk_g2s(sb + L::v_off, p.v4 + tk * (32 * D), 32 * D, &bar_full[st]);
+                        bulk_g2s(sb + L::ksf_off, p.sfk + tk * 512, 512, &bar_full[st]);
+                        bulk_g2s(sb + L::vsf_off, p.sfv + tk * 512, 512, &bar_full[st]);
+                    }
+                    ++loads_issued;
+                }
+            }
+        } else if (warp == 4) {
+            // ================================================== MMA issue
+            if (lane == 0) {
+                bool ok = mbar_wait(&bar_q, nitem & 1, abort_v, p.status);
+                ok = ok && mbar_wait(&bar_sfq, nitem & 1, abort_v, p.status);
+                tc_fence_after();
+                if (ok && n_ent > n8e) {
+                    for (int ch = 0; ch < D / 64; ++ch)
+                        tc_cp_32x128_x4(tmem + kColSfq + 4 * ch, sdesc(smem + L::sfq + 512 * ch, 128, 128));
+                }
+                auto issue_pv = [&](int i) -> bool {
+                    const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
+                    if (!mbar_wait(&bar_p[pb], (g >> 1) & 1, abort_v, p.status)) return false;
+                    tc_fence_after();
+                    const uint32_t e = list[i];
+                    const int ph = (e >> 16) & 1;
+                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                    uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
+                    if (ph == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk)
+                            mma_f8(tmem + kColO, sdesc(pbuf + 256 * kk, 128, 512), sdesc(sb + L::v_off + 256 * kk, 128, 512),
+                                   idesc_f8(128, D), (i > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        tc_cp_32x128_x4(tmem + kColSfp + 4 * pb, sdesc(pbuf + 128 * 64, 128, 128));
+                        tc_cp_32x128_x4(tmem + kColSfv + 4 * pb, sdesc(sb + L::vsf_off, 128, 128));
+                        mma_f4(tmem + kColO, sdesc(pbuf, 128, 256), sdesc(sb + L::v_off, 128, 256), idesc_f4(128, D),
+                               tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bar_empty[st]);
+                    tc_commit(&bar_pv[pb]);
+                    return true;
+                };
+                for (int j = 0; j < n_ent && ok; ++j) {
+                    const uint32_t g = gstep + j, st = g % kStages, sbuf = g & 1;
+                    if (!mbar_wait(&bar_full[st], (g / kStages) & 1, abort_v, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t e = list[j];
+                    const int ph = (e >> 16) & 1;
+                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                    const uint32_t sd = tmem + kColS + 64 * sbuf;
+                    if (ph == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 32; ++kk)
+                            mma_f8(sd, sdesc(smem + L::q8 + 256 * kk, 128, 8 * D), sdesc(sb + L::k_off + 256 * kk, 128, 8 * D),
+                                   idesc_f8(128, 64), kk > 0 ? 1u : 0u);
+                    } else {
+                        tc_cp_32x128_x4(tmem + kColSfk + 4 * sbuf, sdesc(sb + L::ksf_off, 128, 128));
+#pragma unroll
+                        for (int kk = 0; kk < D / 64; ++kk)
+                            mma_f4(sd, sdesc(smem + L::q4 + 256 * kk, 128, 4 * D), sdesc(sb + L::k_off + 256 * kk, 128, 4 * D),
+                                   idesc_f4(128, 64), tmem + kColSfq + 4 * kk, tmem + kColSfk + 4 * sbuf + 2 * kk,
+                                   kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bar_s[sbuf]);
+                    mma_issued = true;
+                    if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+                }
+                if (ok && n_ent > 0) ok = issue_pv(n_ent - 1);
+            }
+        } else {
+            // ================================================== softmax
+            const int r = tid;            // tile row
+            const int hf = r >> 6;        // which query block of the pair
+            const int a = hf ? a1 : a0;
+            const bool qvalid = hf == 0 || has1;
+            const size_t ta = (size_t)bh * R + (qvalid ? a : a0);
+            const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+            const float rd = D == 64 ? 0.125f : 0.0883883461356163025f;  // 1/sqrt(D)
+            const float kLog2e = 1.4426950408889634f;
+            // Q scale factors of this row into the copy atoms (one per 64 channels)
+            {
+                uint8_t* atom = smem + L::sfq;
+                const uint8_t* src = p.sfq + ta * (64 * (D / 16)) + (r & 63) * (D / 16);
+                for (int ch = 0; ch < D / 64; ++ch) {
+                    uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * ch) : 0u;
+                    *reinterpret_cast<uint32_t*>(atom + 512 * ch + 16 * (r & 31) + 4 * (r >> 5)) = w;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&bar_sfq);
+            }
+            const float sq8 = p.scale[ta], gq4 = p.scale[(size_t)3 * BH * R + ta];
+            const float vm8 = p.vmax[bh], vm4 = p.vmax[BH + bh];
+            const float sig8 = __fdiv_rn(vm8, 448.0f), sig4 = __fdiv_rn(vm4, 2688.0f);
+            float m = -INFINITY, l = 0.0f;
+            bool ok = true;
+            for (int j = 0; j < n_ent && ok; ++j) {
+                const uint32_t g = gstep + j, sbuf = g & 1, pb = g & 1;
+                const uint32_t e = list[j];
+                const int kb = e & 0xFFFF, ph = (e >> 16) & 1;
+                const bool active = (e >> (17 + hf)) & 1;
+                const size_t tk = (size_t)bh * R + kb;
+                const int nk = p.n_a[kb];
+                bool waited = mbar_wait(&bar_s[sbuf], (g >> 1) & 1, abort_v, p.status);
+                // P buffer pb was last read by the PV of step g-2
+                if (waited && g >= 2) waited = mbar_wait(&bar_pv[pb], ((g - 2) >> 1) & 1, abort_v, p.status);
+                if (!__all_sync(0xffffffffu, waited)) { ok = false; break; }
+                tc_fence_after();
+                uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
+                float corr = 1.0f;
+                bool resc = false;
+                if (active) {
+                    uint32_t s[64];
+                    tmem_ld32(lane_base + kColS + 64 * sbuf, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+                    tmem_ld32(lane_base + kColS + 64 * sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+                    tc_wait_ld();
+                    const float cs = ph == 0 ? sq8 * p.scale[(size_t)BH * R + tk] : gq4 * p.scale[(size_t)4 * BH * R + tk];
+                    const float c2 = cs * rd * kLog2e;
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        const float v = __uint_as_float(s[c]) * c2;
+                        s[c] = __float_as_uint(c < nk ? v : -INFINITY);
+                        mx = fmaxf(mx, __uint_as_float(s[c]));
+                    }
+                    const float mn = fmaxf(m, mx);
+                    if (m != -INFINITY && mn > m) {
+                        corr = ex2(m - mn);
+                        resc = true;
+                    }
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        const float pv = ex2(__uint_as_float(s[c]) - mn);
+                        s[c] = __float_as_uint(pv);
+                        sum += pv;
+                    }
+                    l = l * corr + sum;
+                    m = mn;
+                    if (ph == 0) {
+                        const float ratio = sig8 > 0.0f ? __fdiv_rn(p.scale[(size_t)2 * BH * R + tk], sig8) : 0.0f;
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const int c = ch * 16 + q * 4;
+                                const uint16_t lo = cvt_e4m3x2(__fmul_rn(__uint_as_float(s[c]), ratio),
+                                                               __fmul_rn(__uint_as_float(s[c + 1]), ratio));
+                                const uint16_t hi = cvt_e4m3x2(__fmul_rn(__uint_as_float(s[c + 2]), ratio),
+                                                               __fmul_rn(__uint_as_float(s[c + 3]), ratio));
+                                w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+                            }
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    } else {
+                        const float ratio = sig4 > 0.0f ? __fdiv_rn(p.scale[(size_t)5 * BH * R + tk], sig4) : 0.0f;
+                        uint32_t sfw = 0;
+#pragma unroll
+                        for (int gi = 0; gi < 4; ++gi) {
+                            float y[16], ym = 0.0f;
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                y[q] = __fmul_rn(__uint_as_float(s[gi * 16 + q]), ratio);
+                                ym = fmaxf(ym, y[q]);
+                            }
+                            const uint8_t sf = (uint8_t)(cvt_e4m3x2(__fdiv_rn(ym, 6.0f), 0.0f) & 0xFF);
+                            const float rc = sf ? __fdiv_rn(1.0f, e4m3_to_f32(sf)) : 0.0f;
+                            uint32_t w[2];
+#pragma unroll
+                            for (int hw = 0; hw < 2; ++hw) {
+                                uint32_t acc = 0;
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const int c = hw * 8 + 2 * q;
+                                    const uint32_t byte = cvt_e2m1x2(__fmul_rn(y[c], rc), __fmul_rn(y[c + 1], rc));
+                                    acc |= byte << (8 * q);
+                                }
+                                w[hw] = sf ? acc : 0u;
+                            }
+                            // 16 keys = 8 bytes: half of a 16-byte chunk
+                            *reinterpret_cast<uint2*>(pbuf + kmajor_off(r, gi >> 1, 32) + 8 * (gi & 1)) =
+                                make_uint2(w[0], w[1]);
+                            sfw |= (uint32_t)sf << (8 * gi);
+                        }
+                        *reinterpret_cast<uint32_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5)) = sfw;
+                    }
+                } else {
+                    // row not in this step: zero weights
+                    if (ph == 0) {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch)
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) = make_uint4(0, 0, 0, 0);
+                    } else {
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch)
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 32)) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint32_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5)) = 0u;
+                    }
+                }
+                // O rescale: when the row max grew, and for every row at the
+                // switch from the 8-bit to the 4-bit phase (units sigma8 -> sigma4).
+                const bool sw = (j == n8e) && (j > 0);
+                float f = corr;
+                if (sw) f *= (sig4 > 0.0f ? __fdiv_rn(sig8, sig4) : 1.0f);
+                const bool need = (resc || sw) && j > 0;
+                if (__any_sync(0xffffffffu, need)) {
+                    // O must hold the PV of step g-1 first
+                    const bool waited = mbar_wait(&bar_pv[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_v, p.status);
+                    if (!__all_sync(0xffffffffu, waited)) ok = false;
+                    if (ok) {
+                        tc_fence_after();
+                        const float fm = need ? f : 1.0f;
+#pragma unroll
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(lane_base + kColO + c0, o);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fm);
+                            tmem_st32(lane_base + kColO + c0, o);
+                        }
+                        tc_wait_st();
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar_p[pb]);
+            }
+            // ---- epilogue
+            ok = __all_sync(0xffffffffu, ok);
+            float o_scale = 0.0f;
+            const bool have = n_ent > 0 && ok;
+            if (have) {
+                const uint32_t g = gstep + n_ent - 1;
+                if (!mbar_wait(&bar_pv[g & 1], (g >> 1) & 1, abort_v, p.status)) ok = false;
+                tc_fence_after();
+                const float unit = n_ent > n8e ? sig4 : sig8;
+                o_scale = l > 0.0f ? __fdiv_rn(unit, l) : 0.0f;
+            }
+            const bool have_o = __all_sync(0xffffffffu, have && ok);
+            const int qrow = r & 63;
+            const bool store = qvalid && qrow < p.n_a[a];
+            __nv_bfloat16* dst = p.out;
+            if (store) {
+                const int t = p.slot_token[a * 64 + qrow];
+                dst += (size_t)(bh / p.H) * p.o0 + (size_t)(bh % p.H) * p.o1 + (size_t)t * p.o2;
+            }
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                if (have_o) {
+                    tmem_ld32(lane_base + kColO + c0, o);
+                    tc_wait_ld();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0u;
+                }
+                if (!store) continue;
+                uint32_t packed[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float x0 = o_scale > 0.0f ? __uint_as_float(o[2 * c]) * o_scale : 0.0f;
+                    const float x1 = o_scale > 0.0f ? __uint_as_float(o[2 * c + 1]) * o_scale : 0.0f;
+                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                    packed[c] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    *reinterpret_cast<uint4*>(dst + c0 + 8 * v) =
+                        make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            }
+        }
+        gstep += n_ent;
+    }
+
+    // ---- teardown: drain outstanding async work, then free tensor memory
+    __syncthreads();
+    if (warp == 4 && lane == 0 && mma_issued) {
+        tc_commit(&bar_drain);
+        for (uint32_t i = 0; i < DA2_WAIT_LIMIT; ++i) {
+            if (mbar_try_wait(&bar_drain, 0)) break;
+            __nanosleep(128);
+        }
+    }
+    if (warp == 5 && lane == 0) {
+        // every issued stage fill must have landed before the CTA exits
+        for (uint32_t k = 0; k < loads_issued && k < (uint32_t)kStages; ++k) {
+            const uint32_t g = loads_issued - 1 - k, st = g % kStages;
+            for (uint32_t i = 0; i < DA2_WAIT_LIMIT; ++i) {
+                if (mbar_try_wait(&bar_full[st], (g / kStages) & 1)) break;
+                __nanosleep(128);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// At least 120 KB so that a single CTA fits on an SM: each CTA holds all 512
+// tensor-memory columns for its lifetime.
+template <int D>
+size_t attention_smem_bytes(int R) {
+    const size_t need = Smem<D>::list + (size_t)2 * R * sizeof(uint32_t);
+    return need > 120 * 1024 ? need : 120 * 1024;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream) {
+    const int items = p.B * p.H * ((p.R + 1) / 2);
+    if (items == 0) return cudaSuccess;
+    const int grid = items < p.num_sms ? items : p.num_sms;
+    cudaError_t e;
+    if (p.d == 64) {
+        const size_t smem = attention_smem_bytes<64>(p.R);
+        e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attention_kernel<64><<<grid, kThreads, smem, stream>>>(p);
+    } else {
+        const size_t smem = attention_smem_bytes<128>(p.R);
+        e = cudaFuncSetAttribute(attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attention_kernel<128><<<grid, kThreads, smem, stream>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace da2

@@ -1,0 +1,71 @@
+// da2_kernels.h -- launch interfaces of the DraftAttention2 kernels (internal).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace da2 {
+
+struct PrepareArgs {
+    int B, H, d, R;
+    const __nv_bfloat16 *q, *k, *v;
+    long long s0, s1, s2;      // element strides of batch, head, token
+    const int32_t* slot_token; // [64 R] token of each slot, -1 = padding
+    const int32_t* n_a;        // [R]
+    double* desc;
+    uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
+    float* scale;
+    float* vmax;
+};
+cudaError_t launch_prepare(const PrepareArgs& p, cudaStream_t stream);
+
+// Per head and per quota target, the state of the radix selection of the
+// T-th largest 96-bit key (A bits : ~pair index).
+struct SelectTarget {
+    unsigned long long p_hi;  // selected prefix, left aligned in 96 bits
+    unsigned int p_lo;
+    int nbits;                // bits of the key already fixed
+    long long need;           // rank still sought inside the current prefix (1-based)
+    int unique;               // the current prefix holds exactly one key: record it next pass
+    int done;                 // threshold known (or no threshold: none)
+    int none;                 // T == 0: nothing gets this precision or better
+    unsigned long long key_hi;
+    unsigned int key_lo;
+};
+
+struct PlanArgs {
+    int BH, R, d;
+    int bp8, bp4;
+    double lambda;
+    const double* desc;      // [4][BH][R][d]
+    double* A;               // [BH][R][R] (first holds the average-branch logits)
+    double* Lmax;            // [BH][R][R] max-branch logits (scratch)
+    unsigned long long* abits_minmax;  // [BH][2] (scratch)
+    SelectTarget* sel;       // [BH][2] (scratch)
+    unsigned int* hist;      // [BH][2][4096] (scratch)
+    uint8_t* prec;           // [BH][R][R]
+    int32_t* cnt;            // [2][BH][R]
+    uint16_t* kidx;          // [BH][R][R]
+    unsigned* status;
+};
+size_t plan_scratch_bytes(int BH, int R);
+void plan_carve_scratch(PlanArgs* p, void* scratch);
+cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream);
+
+struct AttnArgs {
+    int B, H, d, R, N;
+    const int32_t* slot_token;  // [64 R]
+    const int32_t* n_a;         // [R]
+    const uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
+    const float* scale;  // [6][BH][R]
+    const float* vmax;   // [2][BH]
+    const int32_t* cnt;  // [2][BH][R]
+    const uint16_t* kidx;  // [BH][R][R]
+    __nv_bfloat16* out;
+    long long o0, o1, o2;  // element strides of the output
+    unsigned* status;
+    int num_sms;
+};
+cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream);
+
+}  // namespace da2

@@ -1,0 +1,443 @@
+// da2_plan.cu -- draft map and routing ("DraftAttention2", Eq. 3; Sec. 3.1
+// "Joint allocation of sparsity and precision"; App. C.1 "Routing and
+// precision formats").
+//
+// The ranking of all R^2 region pairs of a head must be reproducible bit for
+// bit, so the draft map is computed in fp64 with a fixed operation order:
+//   logit(a,b) = (fma chain over channels c = 0..d-1 in ascending order,
+//                 starting from 0) * (1/sqrt d)
+//   per row and branch: m = max_b logit; e_b = exp_fixed(logit_b - m);
+//                 Z = sum of e_b in ascending b; S_b = e_b / Z
+//   A = fma(lambda, S^max, (1 - lambda) * S^avg)
+// exp_fixed is a Cody-Waite reduction with a two-part ln2 and a degree-13
+// Taylor polynomial in Horner form (fma), scaled by 2^k; results below the
+// normal range are flushed to zero.  The ranking is an exact radix selection
+// of the T8-th and Tkeep-th largest 96-bit keys (A bits : ~pair index), i.e.
+// A descending with ties to the smaller pair index a*R+b, followed by an
+// exact classification and an ordered per-row compaction of the lists.
+#include <cfloat>
+
+#include "da2_common.cuh"
+#include "da2_kernels.h"
+
+namespace da2 {
+
+namespace {
+
+constexpr double kLog2e = 0x1.71547652b82fep+0;   // 1/ln 2
+constexpr double kLn2Hi = 0x1.62e42fee00000p-1;   // ln 2 cut to 32 significant bits
+constexpr double kLn2Lo = 0x1.a39ef35793c76p-33;  // ln 2 - kLn2Hi
+// 1/n! for n = 0..13, correctly rounded
+__constant__ double kInvFact[14] = {
+    0x1.0000000000000p+0,  0x1.0000000000000p+0,  0x1.0000000000000p-1,  0x1.5555555555555p-3,
+    0x1.5555555555555p-5,  0x1.1111111111111p-7,  0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13,
+    0x1.a01a01a01a01ap-16, 0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+    0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+
+__device__ __forceinline__ double exp_fixed(double x) {
+    if (x < -708.0) return 0.0;
+    if (x > 709.0) return __longlong_as_double(0x7ff0000000000000LL);
+    const double k = rint(x * kLog2e);
+    double r = fma(-k, kLn2Hi, x);
+    r = fma(-k, kLn2Lo, r);
+    double p = kInvFact[13];
+#pragma unroll
+    for (int n = 12; n >= 0; --n) p = fma(p, r, kInvFact[n]);
+    // 2^k with k in [-1021, 1023]: the product is a normal number, exact.
+    return p * __longlong_as_double((long long)((int)k + 1023) << 52);
+}
+
+// ---------------------------------------------------------------- logits
+// 64 x 64 output tile of both branches per CTA; each thread owns 4 x 4
+// outputs per branch and accumulates them in ascending channel order.
+template <int D>
+__global__ void __launch_bounds__(256) logits_kernel(PlanArgs p, double rd) {
+    __shared__ double sQa[16][64], sQm[16][64], sKa[16][64], sKm[16][64];
+    const int R = p.R, bh = blockIdx.z;
+    const int a0 = blockIdx.y * 64, b0 = blockIdx.x * 64;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const size_t plane = (size_t)p.BH * R * D;
+    const double* Qa = p.desc + 0 * plane + (size_t)bh * R * D;
+    const double* Qm = p.desc + 1 * plane + (size_t)bh * R * D;
+    const double* Ka = p.desc + 2 * plane + (size_t)bh * R * D;
+    const double* Km = p.desc + 3 * plane + (size_t)bh * R * D;
+    double acc_a[4][4], acc_m[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc_a[i][j] = acc_m[i][j] = 0.0;
+
+    for (int k0 = 0; k0 < D; k0 += 16) {
+        for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+            const int r = i >> 4, c = i & 15;
+            const int ra = a0 + r, rb = b0 + r;
+            sQa[c][r] = ra < R ? Qa[(size_t)ra * D + k0 + c] : 0.0;
+            sQm[c][r] = ra < R ? Qm[(size_t)ra * D + k0 + c] : 0.0;
+            sKa[c][r] = rb < R ? Ka[(size_t)rb * D + k0 + c] : 0.0;
+            sKm[c][r] = rb < R ? Km[(size_t)rb * D + k0 + c] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            double qa[4], qm[4], ka[4], km[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                qa[i] = sQa[c][ty * 4 + i];
+                qm[i] = sQm[c][ty * 4 + i];
+                ka[i] = sKa[c][tx * 4 + i];
+                km[i] = sKm[c][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc_a[i][j] = fma(qa[i], ka[j], acc_a[i][j]);
+                    acc_m[i][j] = fma(qm[i], km[j], acc_m[i][j]);
+                }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int a = a0 + ty * 4 + i;
+        if (a >= R) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int b = b0 + tx * 4 + j;
+            if (b >= R) continue;
+            const size_t o = ((size_t)bh * R + a) * R + b;
+            p.A[o] = acc_a[i][j] * rd;
+            p.Lmax[o] = acc_m[i][j] * rd;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- softmax
+// One CTA per (head, query region): both branches, fixed summation order.
+constexpr int kSoftThreads = 128;
+
+__device__ __forceinline__ double block_max(double v, double* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    double m = red[0];
+#pragma unroll
+    for (int w = 1; w < kSoftThreads / 32; ++w) m = fmax(m, red[w]);
+    __syncthreads();
+    return m;
+}
+
+__global__ void __launch_bounds__(kSoftThreads) softmax_kernel(PlanArgs p) {
+    extern __shared__ double sm[];
+    __shared__ double red[kSoftThreads / 32];
+    __shared__ double Z[2];
+    __shared__ unsigned long long mm[2][kSoftThreads / 32];
+    const int R = p.R;
+    const size_t row = blockIdx.x;
+    const int bh = (int)(row / R);
+    double* la = sm;
+    double* lm = sm + R;
+    double* Arow = p.A + row * R;
+    const double* Mrow = p.Lmax + row * R;
+    double ma = -DBL_MAX, mx = -DBL_MAX;
+    for (int b = threadIdx.x; b < R; b += kSoftThreads) {
+        const double x = Arow[b], y = Mrow[b];
+        la[b] = x;
+        lm[b] = y;
+        ma = fmax(ma, x);
+        mx = fmax(mx, y);
+    }
+    ma = block_max(ma, red);
+    mx = block_max(mx, red);
+    for (int b = threadIdx.x; b < R; b += kSoftThreads) {
+        la[b] = exp_fixed(la[b] - ma);
+        lm[b] = exp_fixed(lm[b] - mx);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 || threadIdx.x == 32) {
+        const double* e = threadIdx.x == 0 ? la : lm;
+        double z = 0.0;
+        for (int b = 0; b < R; ++b) z += e[b];
+        Z[threadIdx.x == 0 ? 0 : 1] = z;
+    }
+    __syncthreads();
+    const double za = Z[0], zm = Z[1];
+    const double lam = p.lambda, oml = 1.0 - p.lambda;
+    unsigned long long lo = ~0ull, hi = 0ull;
+    for (int b = threadIdx.x; b < R; b += kSoftThreads) {
+        const double A = fma(lam, lm[b] / zm, oml * (la[b] / za));
+        Arow[b] = A;
+        const unsigned long long bits = (unsigned long long)__double_as_longlong(A);
+        lo = bits < lo ? bits : lo;
+        hi = bits > hi ? bits : hi;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+        const unsigned long long h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+        lo = l2 < lo ? l2 : lo;
+        hi = h2 > hi ? h2 : hi;
+    }
+    if ((threadIdx.x & 31) == 0) {
+        mm[0][threadIdx.x >> 5] = lo;
+        mm[1][threadIdx.x >> 5] = hi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kSoftThreads / 32; ++w) {
+            lo = mm[0][w] < lo ? mm[0][w] : lo;
+            hi = mm[1][w] > hi ? mm[1][w] : hi;
+        }
+        atomicMin(&p.abits_minmax[bh], lo);
+        atomicMax(&p.abits_minmax[p.BH + bh], hi);
+    }
+}
+
+// ---------------------------------------------------------------- selection
+// Key of pair i of a head: 96 bits = A bits (64) : 0xFFFFFFFF - i (32).
+// Larger key = higher rank (larger A, or equal A and smaller index).
+struct Key {
+    unsigned long long hi;
+    unsigned int lo;
+};
+
+__device__ __forceinline__ void top_mask(int nbits, unsigned long long* mh, unsigned int* ml) {
+    *mh = nbits <= 0 ? 0ull : (nbits >= 64 ? ~0ull : (~0ull << (64 - nbits)));
+    const int nl = nbits - 64;
+    *ml = nl <= 0 ? 0u : (nl >= 32 ? ~0u : (~0u << (32 - nl)));
+}
+
+__device__ __forceinline__ unsigned digit_at(Key k, int pos, int w) {
+    // bits [pos, pos + w) of the 96-bit key, bit 0 = lsb of lo
+    const unsigned mask = (1u << w) - 1u;
+    if (pos >= 32) return (unsigned)(k.hi >> (pos - 32)) & mask;
+    if (pos + w <= 32) return (k.lo >> pos) & mask;
+    return (unsigned)((k.hi << (32 - pos)) | (unsigned long long)(k.lo >> pos)) & mask;
+}
+
+__global__ void select_init_kernel(PlanArgs p, long long T8, long long Tk) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= p.BH) return;
+    const unsigned long long lo = p.abits_minmax[bh], hi = p.abits_minmax[p.BH + bh];
+    const int c = (lo == hi) ? 64 : __clzll((long long)(lo ^ hi));
+    for (int t = 0; t < 2; ++t) {
+        SelectTarget s;
+        s.nbits = c;
+        s.p_hi = (c >= 64) ? lo : (c == 0 ? 0ull : (lo & (~0ull << (64 - c))));
+        s.p_lo = 0u;
+        s.need = t == 0 ? T8 : Tk;
+        s.unique = 0;
+        s.none = s.need == 0;
+        s.done = s.none;
+        s.key_hi = 0ull;
+        s.key_lo = 0u;
+        p.sel[bh * 2 + t] = s;
+    }
+}
+
+constexpr int kHistThreads = 256;
+constexpr int kHistChunk = 16384;
+
+__global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p) {
+    __shared__ unsigned h[2][4096];
+    const int bh = blockIdx.y;
+    SelectTarget s[2] = {p.sel[bh * 2], p.sel[bh * 2 + 1]};
+    if (s[0].done && s[1].done) return;
+    for (int i = threadIdx.x; i < 2 * 4096; i += kHistThreads) (&h[0][0])[i] = 0u;
+    __syncthreads();
+    unsigned long long mh[2];
+    unsigned ml[2];
+    int w[2], pos[2];
+    for (int t = 0; t < 2; ++t) {
+        top_mask(s[t].nbits, &mh[t], &ml[t]);
+        w[t] = min(12, 96 - s[t].nbits);
+        pos[t] = 96 - s[t].nbits - w[t];
+    }
+    const size_t RR = (size_t)p.R * p.R;
+    const size_t begin = (size_t)blockIdx.x * kHistChunk;
+    const size_t end = min(begin + (size_t)kHistChunk, RR);
+    const double* Ah = p.A + (size_t)bh * RR;
+    for (size_t i = begin + threadIdx.x; i < end; i += kHistThreads) {
+        Key k;
+        k.hi = (unsigned long long)__double_as_longlong(Ah[i]);
+        k.lo = 0xFFFFFFFFu - (unsigned)i;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (s[t].done) continue;
+            if (((k.hi ^ s[t].p_hi) & mh[t]) || ((k.lo ^ s[t].p_lo) & ml[t])) continue;
+            if (s[t].unique) {
+                p.sel[bh * 2 + t].key_hi = k.hi;
+                p.sel[bh * 2 + t].key_lo = k.lo;
+                p.sel[bh * 2 + t].done = 1;
+            } else {
+                atomicAdd(&h[t][digit_at(k, pos[t], w[t])], 1u);
+            }
+        }
+    }
+    __syncthreads();
+    unsigned* gh = p.hist + (size_t)bh * 2 * 4096;
+    for (int i = threadIdx.x; i < 2 * 4096; i += kHistThreads) {
+        const unsigned v = (&h[0][0])[i];
+        if (v) atomicAdd(&gh[i], v);
+    }
+}
+
+// One warp per (head, target): choose the digit holding the sought rank.
+__global__ void __launch_bounds__(64) select_scan_kernel(PlanArgs p) {
+    const int bh = blockIdx.x, t = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned* gh = p.hist + ((size_t)bh * 2 + t) * 4096;
+    SelectTarget* sp = &p.sel[bh * 2 + t];
+    SelectTarget s = *sp;
+    if (!s.done && !s.unique) {
+        const int w = min(12, 96 - s.nbits), pos = 96 - s.nbits - w;
+        // lane covers bins [4095 - 128 lane - 127, 4095 - 128 lane], descending
+        const int top = 4095 - 128 * lane;
+        unsigned long long sum = 0;
+        for (int i = 0; i < 128; ++i) sum += gh[top - i];
+        unsigned long long incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const unsigned long long excl = incl - sum;
+        const bool mine = (long long)excl < s.need && s.need <= (long long)incl;
+        if (mine) {
+            long long cum = (long long)excl;
+            for (int i = 0; i < 128; ++i) {
+                const int bin = top - i;
+                const long long c = gh[bin];
+                if (cum + c >= s.need) {
+                    s.need -= cum;
+                    if (pos >= 32) s.p_hi |= (unsigned long long)bin << (pos - 32);
+                    else {
+                        s.p_lo |= (unsigned)bin << pos;
+                        if (pos + w > 32) s.p_hi |= (unsigned long long)bin >> (32 - pos);
+                    }
+                    s.nbits += w;
+                    if (s.nbits >= 96) {
+                        s.done = 1;
+                        s.key_hi = s.p_hi;
+                        s.key_lo = s.p_lo;
+                    } else if (c == 1) {
+                        s.unique = 1;
+                    }
+                    *sp = s;
+                    break;
+                }
+                cum += c;
+            }
+        }
+    }
+    __syncwarp();
+    for (int i = lane; i < 4096; i += 32) gh[i] = 0u;
+}
+
+// ---------------------------------------------------------------- classify
+// One warp per (head, query region): precision of every pair, then the
+// ordered list of 8-bit key blocks followed by the 4-bit key blocks.
+__global__ void __launch_bounds__(128) classify_kernel(PlanArgs p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t row = (size_t)blockIdx.x * 4 + warp;
+    const int R = p.R;
+    if (row >= (size_t)p.BH * R) return;
+    const int bh = (int)(row / R), a = (int)(row % R);
+    const SelectTarget s8 = p.sel[bh * 2], sk = p.sel[bh * 2 + 1];
+    const double* Arow = p.A + row * R;
+    uint8_t* prow = p.prec + row * R;
+    uint16_t* krow = p.kidx + row * R;
+    const unsigned lt = (1u << lane) - 1u;
+    auto ge = [](Key k, const SelectTarget& s) {
+        return !s.none && (k.hi > s.key_hi || (k.hi == s.key_hi && k.lo >= s.key_lo));
+    };
+    int n8 = 0;
+    for (int b0 = 0; b0 < R; b0 += 32) {
+        const int b = b0 + lane;
+        bool is8 = false;
+        if (b < R) {
+            Key k;
+            k.hi = (unsigned long long)__double_as_longlong(Arow[b]);
+            k.lo = 0xFFFFFFFFu - (unsigned)(a * R + b);
+            is8 = ge(k, s8);
+            const bool keep = ge(k, sk);
+            prow[b] = is8 ? 8 : (keep ? 4 : 0);
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, is8);
+        if (is8) krow[n8 + __popc(m & lt)] = (uint16_t)b;
+        n8 += __popc(m);
+    }
+    __syncwarp();
+    int n4 = 0;
+    for (int b0 = 0; b0 < R; b0 += 32) {
+        const int b = b0 + lane;
+        const bool is4 = b < R && prow[b] == 4;
+        const unsigned m = __ballot_sync(0xffffffffu, is4);
+        if (is4) krow[n8 + n4 + __popc(m & lt)] = (uint16_t)b;
+        n4 += __popc(m);
+    }
+    if (lane == 0) {
+        p.cnt[row] = n8;
+        p.cnt[(size_t)p.BH * R + row] = n4;
+    }
+}
+
+constexpr int kSelectPasses = 8;  // 12-bit digits cover the 96-bit key
+
+}  // namespace
+
+size_t plan_scratch_bytes(int BH, int R) {
+    size_t b = (size_t)BH * R * R * sizeof(double);        // max-branch logits
+    b += (size_t)2 * BH * sizeof(unsigned long long);      // A bit range per head
+    b = (b + 255) & ~(size_t)255;
+    b += (size_t)2 * BH * sizeof(SelectTarget);
+    b = (b + 255) & ~(size_t)255;
+    b += (size_t)2 * BH * 4096 * sizeof(unsigned);
+    return b;
+}
+
+void plan_carve_scratch(PlanArgs* p, void* scratch) {
+    char* c = static_cast<char*>(scratch);
+    p->Lmax = reinterpret_cast<double*>(c);
+    size_t off = (size_t)p->BH * p->R * p->R * sizeof(double);
+    p->abits_minmax = reinterpret_cast<unsigned long long*>(c + off);
+    off += (size_t)2 * p->BH * sizeof(unsigned long long);
+    off = (off + 255) & ~(size_t)255;
+    p->sel = reinterpret_cast<SelectTarget*>(c + off);
+    off += (size_t)2 * p->BH * sizeof(SelectTarget);
+    off = (off + 255) & ~(size_t)255;
+    p->hist = reinterpret_cast<unsigned*>(c + off);
+}
+
+cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
+    const int R = p.R, BH = p.BH;
+    const long long RR = (long long)R * R;
+    const long long T8 = RR * p.bp8 / 10000, Tk = RR * (p.bp8 + p.bp4) / 10000;
+    cudaError_t e;
+    const double rd = 1.0 / sqrt((double)p.d);
+    dim3 lg((R + 63) / 64, (R + 63) / 64, BH);
+    if (p.d == 64) logits_kernel<64><<<lg, 256, 0, stream>>>(p, rd);
+    else logits_kernel<128><<<lg, 256, 0, stream>>>(p, rd);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.abits_minmax, 0xFF, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.abits_minmax + BH, 0, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.hist, 0, sizeof(unsigned) * 2 * 4096 * (size_t)BH, stream)) != cudaSuccess) return e;
+    const size_t smem = sizeof(double) * 2 * R;
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(softmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    softmax_kernel<<<(unsigned)((size_t)BH * R), kSoftThreads, smem, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    select_init_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(p, T8, Tk);
+    dim3 hg((unsigned)((RR + kHistChunk - 1) / kHistChunk), BH);
+    for (int pass = 0; pass < kSelectPasses; ++pass) {
+        select_hist_kernel<<<hg, kHistThreads, 0, stream>>>(p);
+        select_scan_kernel<<<BH, 64, 0, stream>>>(p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    classify_kernel<<<(unsigned)(((size_t)BH * R + 3) / 4), 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace da2

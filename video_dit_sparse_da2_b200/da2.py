@@ -1,0 +1,202 @@
+"""Python binding of libda2 (include/da2.h): argument marshalling only.
+
+Every step of the hot path runs in the CUDA kernels behind the C ABI;
+PyTorch supplies device memory and streams.  Importing this module loads the
+in-tree ``libda2.so`` and raises if it is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libda2.so")
+
+OK, ERR_ARG, ERR_ARCH, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
+
+# Every symbol include/da2.h declares.
+EXPORTS = ("da2_create", "da2_destroy", "da2_partition", "da2_sizes", "da2_tables", "da2_prepare", "da2_plan", "da2_attention",
+           "da2_check_device_status", "da2_status_string", "da2_last_cuda_error")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("F", ctypes.c_int),
+                ("Hv", ctypes.c_int), ("Wv", ctypes.c_int), ("C", ctypes.c_int)]
+
+
+class Budget(ctypes.Structure):
+    _fields_ = [("bp_fp8", ctypes.c_int), ("bp_fp4", ctypes.c_int), ("lam", ctypes.c_double)]
+
+
+_SIZE_FIELDS = ("desc", "q8", "k8", "v8", "q4", "k4", "v4", "sfq", "sfk", "sfv", "scale", "vmax",
+                "prec", "cnt", "kidx", "A", "plan_scratch")
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_int), ("Rf", ctypes.c_int), ("Npad", ctypes.c_int)] + \
+               [(f, ctypes.c_size_t) for f in _SIZE_FIELDS]
+
+
+_PREP_FIELDS = ("desc", "q8", "k8", "v8", "q4", "k4", "v4", "sfq", "sfk", "sfv", "scale", "vmax")
+_PLAN_FIELDS = ("prec", "cnt", "kidx", "A", "scratch")
+
+
+class PreparedPtrs(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in _PREP_FIELDS]
+
+
+class PlanPtrs(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in _PLAN_FIELDS]
+
+
+class DA2Error(RuntimeError):
+    pass
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libda2 (raises when the CUDA library has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise DA2Error(f"CUDA library not built: {LIB_PATH} is missing (run __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        L.da2_create.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(P)]
+        L.da2_destroy.argtypes = [P]
+        L.da2_partition.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+        L.da2_sizes.argtypes = [P, ctypes.POINTER(Sizes)]
+        L.da2_tables.argtypes = [P, P, P]
+        L.da2_prepare.argtypes = [P, P, P, P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(PreparedPtrs), P]
+        L.da2_plan.argtypes = [P, ctypes.POINTER(PreparedPtrs), ctypes.POINTER(Budget), ctypes.POINTER(PlanPtrs), P]
+        L.da2_attention.argtypes = [P, ctypes.POINTER(PreparedPtrs), ctypes.POINTER(PlanPtrs), P,
+                                    ctypes.POINTER(ctypes.c_int64), P]
+        L.da2_check_device_status.argtypes = [P, P]
+        L.da2_status_string.restype = ctypes.c_char_p
+        L.da2_status_string.argtypes = [ctypes.c_int]
+        L.da2_last_cuda_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        msg = lib().da2_status_string(rc).decode()
+        if rc == ERR_CUDA:
+            msg += ": " + lib().da2_last_cuda_error().decode()
+        raise DA2Error(f"{what} failed: {msg} ({rc})")
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _strides(t: torch.Tensor):
+    return (ctypes.c_int64 * 4)(*t.stride())
+
+
+@dataclass
+class Prepared:
+    """Caller-owned prepared operands (uint8 device tensors, layouts in da2.h)."""
+    bufs: dict
+
+    def ptrs(self) -> PreparedPtrs:
+        return PreparedPtrs(**{f: self.bufs[f].data_ptr() for f in _PREP_FIELDS})
+
+
+@dataclass
+class Plan:
+    bufs: dict
+
+    def ptrs(self) -> PlanPtrs:
+        return PlanPtrs(**{f: self.bufs[f].data_ptr() for f in _PLAN_FIELDS})
+
+
+def partition(F: int, Hv: int, Wv: int):
+    """Host partition of a shape: (slot_token[64 R], n_a[R]) as numpy int32 arrays."""
+    import numpy as np
+    R = F * (-(-(Hv * Wv) // 64))
+    st = np.zeros(64 * R, np.int32)
+    na = np.zeros(R, np.int32)
+    rc = lib().da2_partition(F, Hv, Wv, st.ctypes.data_as(ctypes.c_void_p), na.ctypes.data_as(ctypes.c_void_p))
+    if rc != R:
+        _check(rc if rc < 0 else ERR_ARG, "da2_partition")
+    return st, na
+
+
+class DA2:
+    """One shape: its partition tables and helpers to run the three steps."""
+
+    def __init__(self, B: int, H: int, d: int, F: int, Hv: int, Wv: int):
+        self.shape = Shape(B, H, d, F, Hv, Wv, 64)
+        h = ctypes.c_void_p()
+        _check(lib().da2_create(ctypes.byref(self.shape), ctypes.byref(h)), "da2_create")
+        self.handle = h
+        self.sizes = Sizes()
+        _check(lib().da2_sizes(h, ctypes.byref(self.sizes)), "da2_sizes")
+        self.R, self.Npad = self.sizes.R, self.sizes.Npad
+
+    def close(self):
+        if self.handle:
+            lib().da2_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def tables(self):
+        import numpy as np
+        st = np.zeros(self.Npad, np.int32)
+        na = np.zeros(self.R, np.int32)
+        _check(lib().da2_tables(self.handle, st.ctypes.data_as(ctypes.c_void_p), na.ctypes.data_as(ctypes.c_void_p)),
+               "da2_tables")
+        return st, na
+
+    def _alloc(self, fields, device):
+        return {f: torch.empty(max(int(getattr(self.sizes, f if f != "scratch" else "plan_scratch")), 16),
+                               dtype=torch.uint8, device=device) for f in fields}
+
+    def alloc_prepared(self, device="cuda") -> Prepared:
+        return Prepared(self._alloc(_PREP_FIELDS, device))
+
+    def alloc_plan(self, device="cuda") -> Plan:
+        return Plan(self._alloc(_PLAN_FIELDS, device))
+
+    def prepare(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, prep: Prepared, stream=None):
+        assert q.dtype == k.dtype == v.dtype == torch.bfloat16
+        assert q.stride() == k.stride() == v.stride()
+        _check(lib().da2_prepare(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), _strides(q),
+                                 ctypes.byref(prep.ptrs()), _stream_ptr(stream)), "da2_prepare")
+
+    def plan(self, prep: Prepared, plan: Plan, bp8: int, bp4: int, lam: float = 0.2, stream=None):
+        b = Budget(int(bp8), int(bp4), float(lam))
+        _check(lib().da2_plan(self.handle, ctypes.byref(prep.ptrs()), ctypes.byref(b), ctypes.byref(plan.ptrs()),
+                              _stream_ptr(stream)), "da2_plan")
+
+    def attention(self, prep: Prepared, plan: Plan, out: torch.Tensor, stream=None):
+        assert out.dtype == torch.bfloat16
+        _check(lib().da2_attention(self.handle, ctypes.byref(prep.ptrs()), ctypes.byref(plan.ptrs()),
+                                   out.data_ptr(), _strides(out), _stream_ptr(stream)), "da2_attention")
+
+    def check_status(self, stream=None):
+        _check(lib().da2_check_device_status(self.handle, _stream_ptr(stream)), "device status")
+
+    def forward(self, q, k, v, bp8, bp4, lam=0.2, out=None, prep=None, plan=None, stream=None):
+        """prepare -> plan -> attention; returns (out, prep, plan)."""
+        prep = prep or self.alloc_prepared(q.device)
+        plan = plan or self.alloc_plan(q.device)
+        out = torch.empty_like(q) if out is None else out
+        self.prepare(q, k, v, prep, stream)
+        self.plan(prep, plan, bp8, bp4, lam, stream)
+        self.attention(prep, plan, out, stream)
+        return out, prep, plan
