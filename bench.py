@@ -1,0 +1,334 @@
+"""Benchmark of the DraftAttention2 hot path on B200: prepare -> plan -> attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path (fused preparation, draft-guided
+routing, phased FP8/NVFP4 attention) over one synthetic batch already
+resident in HBM.  Prints one JSON line (rank 0).  Multi-GPU: one process per
+GPU (torchrun); every rank runs its own independent call (heads and batches
+are independent problems), no data-path collective, weak scaling; time is
+the max over ranks.
+
+--impl reference times the float64 CPU oracle (the correctness reference of
+this repository) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call and dense-equiv TFLOPS at 1 B200; % of mixed FP8/FP4 tensor roofline"
+UNIT = "TFLOPS (dense-equivalent, whole job)"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+                "bf16_tflops_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def dense_equiv_flops(w) -> float:
+    return 4.0 * w.B * w.H * w.N * w.N * w.d
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+def kept_pair_counts(plan_cnt, B, H, R):
+    """(#FP8 pairs, #NVFP4 pairs) from the plan's per-row counts."""
+    import torch
+    c = plan_cnt[: 2 * B * H * R * 4].view(torch.int32).reshape(2, -1).to(torch.int64)
+    return int(c[0].sum().item()), int(c[1].sum().item())
+
+
+def run_ours(args, w, rank, world):
+    import torch
+
+    from video_dit_sparse_da2_b200 import da2
+    from video_dit_sparse_da2_b200.inputs import workload_qkv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    m = da2.DA2(w.B, w.H, w.d, w.F, w.Hv, w.Wv)
+    qh, kh, vh = (t.pin_memory() for t in workload_qkv(w, seed=0))
+    q, k, v = (t.to(dev) for t in (qh, kh, vh))
+    prep = m.alloc_prepared(dev)
+    plan = m.alloc_plan(dev)
+    out = torch.empty_like(q)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        m.prepare(q, k, v, prep, stream)
+        if ev:
+            ev[1].record(stream)
+        m.plan(prep, plan, w.bp8, w.bp4, w.lam, stream)
+        if ev:
+            ev[2].record(stream)
+        m.attention(prep, plan, out, stream)
+        if ev:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    m.check_status(stream)
+    n8, n4 = kept_pair_counts(plan.bufs["cnt"], w.B, w.H, m.R)
+
+    # ---- device-timed region: inputs resident in HBM
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = Clocks(dev.index)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            step(evs[i])
+    t_end.record(stream)
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    m.check_status(stream)
+    total_ms = t_start.elapsed_time(t_end)
+    per = {"prepare": [], "plan": [], "attention": []}
+    for e in evs:
+        per["prepare"].append(e[0].elapsed_time(e[1]))
+        per["plan"].append(e[1].elapsed_time(e[2]))
+        per["attention"].append(e[2].elapsed_time(e[3]))
+
+    # ---- end to end through the C ABI with host buffers
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+    e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    barrier()
+
+    vals = torch.tensor([total_ms, e2e_ms] + [sum(per[k]) for k in ("prepare", "plan", "attention")],
+                        dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms, t_prep, t_plan, t_attn = vals.tolist()
+    m.close()
+    return dict(total_ms=total_ms, e2e_ms=e2e_ms, t_prep=t_prep / args.steps, t_plan=t_plan / args.steps,
+                t_attn=t_attn / args.steps, n8=n8, n4=n4, R=m.R, clocks=clk,
+                h2d=3 * q.numel() * 2, d2h=out.numel() * 2)
+
+
+def oracle_sample(w, budget_s: float = 20.0):
+    """Time the oracle on a bounded sample of one call of workload w.
+
+    Sample: prepare + draft + assign for `hs` heads (all heads when cheap),
+    attention for a fixed set of query blocks of those heads; the per-call
+    time is extrapolated linearly to all heads and blocks."""
+    import numpy as np
+
+    from oracle import oracle as O
+    from video_dit_sparse_da2_b200.inputs import make_qkv
+
+    cores = O.num_threads()
+    hs = max(1, min(w.H, cores))
+    q, k, v = make_qkv(w.B, hs, w.N, w.d, seed=0)
+    t0 = time.perf_counter()
+    prep = O.prepare(q, k, v, w.F, w.Hv, w.Wv)
+    A = O.draft(prep.desc, w.lam)
+    plan = O.assign(A, w.bp8, w.bp4)
+    t_pp = time.perf_counter() - t0
+    R = A.shape[-1]
+    nblk = 1
+    total_blocks = 0
+    t_att = 0.0
+    sel_all = np.zeros((w.B, hs, R), np.uint8)
+    rng = np.random.default_rng(0)
+    while True:
+        sel = np.zeros((w.B, hs, R), np.uint8)
+        for h in range(hs):
+            sel[0, h, rng.choice(R, size=min(nblk, R), replace=False)] = 1
+        t1 = time.perf_counter()
+        O.attention(q, k, v, w.F, w.Hv, w.Wv, prep, plan, blocks=sel)
+        dt = time.perf_counter() - t1
+        t_att += dt
+        total_blocks += int(sel.sum())
+        sel_all |= sel
+        if t_pp + t_att > budget_s or nblk >= R or dt * 4 > budget_s:
+            break
+        nblk *= 2
+    per_block = t_att / total_blocks * hs  # seconds per block with hs blocks running in parallel threads
+    t_call = (t_pp * w.H / hs) + per_block * R * w.H / hs
+    sample = (f"oracle (C, fp64, OpenMP {cores} threads): prepare+draft+assign on {hs} of {w.H} heads "
+              f"({t_pp:.1f} s), attention on {total_blocks} of {w.H * R} query blocks ({t_att:.1f} s); "
+              f"per-call time extrapolated linearly to all heads and blocks: {t_call:.1f} s")
+    return t_call, cores, sample
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="wan2.1-1.3b-480p")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from video_dit_sparse_da2_b200.inputs import BY_NAME
+    w = BY_NAME[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    flops = dense_equiv_flops(w)
+    config = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "frames": w.F, "latent_hw": [w.Hv, w.Wv],
+              "N": w.N, "budget_fp8_fp4_skip_pct": [w.bp8 / 100, w.bp4 / 100, 100 - (w.bp8 + w.bp4) / 100],
+              "lambda": w.lam, "global_batch": w.B * world, "seq_len": w.N,
+              "parallelism": f"replicas x{world} (independent calls, no collective)",
+              "l2": f"inputs larger than L2 ({3 * w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB of bf16 Q/K/V read per step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        t_call, cores, sample = oracle_sample(w, budget_s=20.0)
+        value = flops / t_call / 1e12
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_call * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
+                "config": config,
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    r = run_ours(args, w, rank, world)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = _peaks()
+    ms = r["total_ms"] / args.steps
+    value = world * flops / (ms * 1e-3) / 1e12
+    # attention roofline: kept-tile FLOPs at the FP8 / FP4 tensor peaks
+    f_pair = 4.0 * 64 * 64 * w.d
+    F8, F4 = r["n8"] * f_pair, r["n4"] * f_pair
+    p8 = 2.0 * peaks["bf16_tflops"] * 1e12   # nominal FP8 : BF16 ratio 2
+    p4 = 4.0 * peaks["bf16_tflops"] * 1e12   # nominal FP4 : BF16 ratio 4
+    t_roof = F8 / p8 + F4 / p4
+    t_att = r["t_attn"] * 1e-3
+    achieved = (F8 + F4) / t_att / 1e12
+    peak_mix = (F8 + F4) / t_roof / 1e12 if t_roof > 0 else None
+    launches_per_step = 1 + (1 + 1 + 1 + 2 * 8 + 1) + 1
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 + nvfp4-e2m1 MMAs (bf16 in/out, fp64 draft)", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": config,
+        "ms_per_call": {"prepare": r["t_prep"], "plan": r["t_plan"], "attention": r["t_attn"], "total": ms},
+        "roofline": {"bound": "tensor", "kernel": "attention", "achieved": achieved, "peak": peak_mix,
+                     "unit": "TFLOP/s", "frac": achieved / peak_mix if peak_mix else None, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TF x2 (FP8) / x4 (NVFP4), "
+                                    f"mixed by the kept FP8/NVFP4 FLOPs",
+                     "fp8_tflop": F8 / 1e12, "fp4_tflop": F4 / 1e12},
+        "prepare_hbm": {"algorithmic_gb": None},
+        "clocks": r["clocks"],
+        "e2e": {"value": world * flops / (r["e2e_ms"] / args.steps * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "ms_per_step": r["e2e_ms"] / args.steps},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    # prepare: algorithmic bytes = bf16 Q/K/V read + every prepared output written once
+    BH, R, d, N = w.B * w.H, r["R"], w.d, w.N
+    prep_bytes = 3 * BH * N * d * 2 + 3 * BH * R * (64 * d + 32 * d) + BH * R * (64 * d // 16 + 2 * 512) \
+        + 4 * BH * R * d * 8 + 6 * BH * R * 4
+    line["prepare_hbm"] = {"algorithmic_gb": prep_bytes / 1e9,
+                           "achieved_gbs": prep_bytes / (r["t_prep"] * 1e-3) / 1e9,
+                           "peak_gbs": peaks["hbm_gbs"],
+                           "frac": prep_bytes / (r["t_prep"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    if world == 1 and not args.no_cpu_baseline:
+        t_call, cores, sample = oracle_sample(w, budget_s=20.0)
+        line["cpu_baseline"] = {"value": flops / t_call / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
