@@ -23,6 +23,8 @@
  *     its partition tables (allocated by da2_create, freed by da2_destroy).
  *   - All device work is asynchronous on the given stream; the call returns
  *     after enqueueing.  A stream of 0 means the legacy default stream.
+ *     Calls on one handle must be ordered (same stream, or synchronized):
+ *     the handle's small device work counter is shared by its launches.
  *   - Return value: DA2_OK or a negative DA2_ERR_* code; nothing is enqueued
  *     when an argument check fails.  DA2_ERR_CUDA means a launch failed; the
  *     CUDA error string is available from da2_last_cuda_error().

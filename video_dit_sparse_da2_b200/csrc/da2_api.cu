@@ -18,6 +18,7 @@ struct da2_ctx {
     int32_t* d_slot_token = nullptr;       // [Npad]
     int32_t* d_n_a = nullptr;              // [R]
     unsigned* d_status = nullptr;          // kernel status word
+    int* d_work = nullptr;                 // attention work counter
 };
 
 namespace {
@@ -103,6 +104,7 @@ int da2_create(const da2_shape* s, da2_handle* out) {
     if ((e = cudaMalloc(&h->d_slot_token, sizeof(int32_t) * h->Npad)) != cudaSuccess ||
         (e = cudaMalloc(&h->d_n_a, sizeof(int32_t) * h->R)) != cudaSuccess ||
         (e = cudaMalloc(&h->d_status, sizeof(unsigned))) != cudaSuccess ||
+        (e = cudaMalloc(&h->d_work, sizeof(int))) != cudaSuccess ||
         (e = cudaMemcpy(h->d_slot_token, h->slot_token.data(), sizeof(int32_t) * h->Npad, cudaMemcpyHostToDevice)) !=
             cudaSuccess ||
         (e = cudaMemcpy(h->d_n_a, h->n_a.data(), sizeof(int32_t) * h->R, cudaMemcpyHostToDevice)) != cudaSuccess ||
@@ -136,6 +138,7 @@ int da2_destroy(da2_handle h) {
     cudaFree(h->d_slot_token);
     cudaFree(h->d_n_a);
     cudaFree(h->d_status);
+    cudaFree(h->d_work);
     delete h;
     return DA2_OK;
 }
@@ -247,6 +250,7 @@ int da2_attention(da2_handle h, const da2_prepared* prep, const da2_plan_bufs* p
     a.o1 = out_strides[1];
     a.o2 = out_strides[2];
     a.status = h->d_status;
+    a.work_counter = h->d_work;
     a.num_sms = h->num_sms;
     cudaError_t e = da2::launch_attention(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DA2_OK : cuda_fail(e);

@@ -11,19 +11,22 @@
 // block kept that key block at that precision, so every row sees exactly its
 // own list in the order of the method.
 //
-// Roles (192 threads, persistent CTAs, one per SM):
+// Roles (192 threads; two persistent CTAs per SM, each holding 256 of the
+// 512 tensor-memory columns; items fetched from a global counter):
 //   warps 0-3  softmax: thread r owns row r of the tile.  Reads S from tensor
-//              memory, keeps the row max m and the unquantized denominator l
-//              (App. B.3), quantizes the weights (FP8: e4m3 of p times the
-//              value-tile scale over the phase unit; NVFP4: the same product
-//              quantized per 16 keys with an e4m3 scale) into shared memory,
-//              rescales its row of O when m grows and once at the phase
-//              switch (sigma8 -> sigma4, the change of units of Eq. 8), and
-//              in the epilogue divides by l, converts to bf16 and stores the
-//              row at its original token position.
+//              memory (then releases the S buffer at once), keeps the row max
+//              m and the unquantized denominator l (App. B.3), quantizes the
+//              weights into shared memory -- FP8: e4m3 of p times the value
+//              tile scale over the phase unit; NVFP4: that product quantized
+//              per 16 keys with a ue4m3 scale -- with the same fp32 rounding
+//              steps as the definition (p of the winning key is exactly 1),
+//              rescales its row of O when m grows and once at the phase switch
+//              (sigma8 -> sigma4, the change of units of Eq. 8), and in the
+//              epilogue divides by l, converts to bf16 and stores the row at
+//              its original token position.
 //   warp 4     MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
-//              kind::mxf4nvf4 block16) into one of two S buffers in tensor
-//              memory, then O += P V into the single O accumulator.
+//              kind::mxf4nvf4 block16) into the S buffer, O += P V into the
+//              single O accumulator.
 //   warp 5     loader (one thread): bulk async copies of the K / V tiles
 //              (pre-tiled by the preparation kernel) into a 3-stage ring.
 // Every mbarrier wait is bounded; a stuck wait sets the status word, all
@@ -39,25 +42,18 @@ namespace {
 constexpr int kStages = 3;
 constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
-constexpr uint32_t kTmemCols = 512;
-// tensor-memory column map
-constexpr uint32_t kColO = 0;       // O accumulator, D columns
-constexpr uint32_t kColS = 128;     // two S buffers of 64 columns
-constexpr uint32_t kColSfq = 256;   // Q scale factors, 4 columns per 64-channel chunk
-constexpr uint32_t kColSfk = 264;   // K scale factors, 2 buffers x 4 columns
-constexpr uint32_t kColSfp = 272;   // P scale factors, 2 buffers x 4 columns
-constexpr uint32_t kColSfv = 280;   // V scale factors, 2 buffers x 4 columns
+constexpr uint32_t kTmemCols = 256;
+// tensor-memory column map (per CTA)
+constexpr uint32_t kColO = 0;      // O accumulator, D columns
+constexpr uint32_t kColS = 128;    // S buffer, 64 columns
+constexpr uint32_t kColSfq = 192;  // Q scale factors, 4 columns per 64-channel chunk
+constexpr uint32_t kColSfk = 200;  // K scale factors, 4 columns
+constexpr uint32_t kColSfp = 204;  // P scale factors, 2 buffers x 4 columns
+constexpr uint32_t kColSfv = 212;  // V scale factors, 2 buffers x 4 columns
 
-struct Entry {  // one step of the merged list
-    static __device__ __forceinline__ uint32_t make(int kb, int phase, int mask) {
-        return (uint32_t)kb | ((uint32_t)phase << 16) | ((uint32_t)mask << 17);
-    }
-};
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
+// Step of the merged list: key block (12 bits), phase (1), row mask (2).
+__device__ __forceinline__ uint16_t make_entry(int kb, int phase, int mask) {
+    return (uint16_t)(kb | (phase << 12) | (mask << 13));
 }
 
 __device__ __forceinline__ uint32_t kmajor_off(int row, int chunk, int row_bytes) {
@@ -76,26 +72,48 @@ struct Smem {
     static constexpr uint32_t p = stage + kStages * stage_bytes;  // 2 x (128 x 64 + 512)
     static constexpr uint32_t p_bytes = 128 * 64 + 512;
     static constexpr uint32_t bitmap = p + 2 * p_bytes;        // 4 x 128 words
-    static constexpr uint32_t list = bitmap + 4 * 128 * 4;     // entries
+    static constexpr uint32_t list = bitmap + 4 * 128 * 4;     // 2R entries of 16 bits
 };
 
+// Per-step scalars of a row: key-block size, score scale, value-scale ratio.
+struct StepMeta {
+    int nk;
+    float ck;     // K tile scale (FP8) or NVFP4 tile scale
+    float ratio;  // V tile scale over the phase unit
+};
+
+__device__ __forceinline__ float rowmax64(const uint32_t (&s)[64]) {
+    float t[22];
+#pragma unroll
+    for (int i = 0; i < 21; ++i)
+        t[i] = max3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]), __uint_as_float(s[3 * i + 2]));
+    t[21] = __uint_as_float(s[63]);
+    float u[8];
+#pragma unroll
+    for (int i = 0; i < 7; ++i) u[i] = max3f(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+    u[7] = t[21];
+    const float v0 = max3f(u[0], u[1], u[2]), v1 = max3f(u[3], u[4], u[5]);
+    return max3f(v0, v1, fmaxf(u[6], u[7]));
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
+__global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
     using L = Smem<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s[2], bar_p[2], bar_pv[2],
-        bar_drain;
+    __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
+        bar_pv[2], bar_drain;
     __shared__ uint32_t tmem_base_sh;
-    __shared__ int abort_sh;
+    __shared__ int abort_sh, item_sh;
     __shared__ int n_ent_sh[2];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int R = p.R, BH = p.B * p.H;
+    const size_t BHR = (size_t)BH * R;
     const int pairs = (R + 1) / 2;
     const int items = BH * pairs;
     const int nwords = (R + 31) / 32;
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + L::bitmap);
-    uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::list);
+    uint16_t* list = reinterpret_cast<uint16_t*>(smem + L::list);
     volatile int* abort_v = &abort_sh;
 
     if (tid == 0) {
@@ -105,8 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
             mbar_init(&bar_full[s], 1);
             mbar_init(&bar_empty[s], 1);
         }
+        mbar_init(&bar_s, 1);
+        mbar_init(&bar_sfree, kSoftmaxThreads);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar_s[s], 1);
             mbar_init(&bar_p[s], kSoftmaxThreads);
             mbar_init(&bar_pv[s], 1);
         }
@@ -123,14 +142,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    uint32_t gstep = 0;  // entries processed by this CTA before the current item
-    uint32_t nitem = 0;  // items processed by this CTA
+    uint32_t gstep = 0;         // steps processed by this CTA before the current item
+    uint32_t nitem = 0;         // items processed by this CTA
     uint32_t loads_issued = 0;  // loader: stage fills issued (for the final drain)
     bool mma_issued = false;
 
-    for (int item = blockIdx.x; item < items; item += gridDim.x, ++nitem) {
+    for (;;) {
+        if (tid == 0) item_sh = atomicAdd(p.work_counter, 1);
         __syncthreads();
-        if (*abort_v) break;
+        const int item = item_sh;
+        if (item >= items || *abort_v) break;
         const int bh = item / pairs, pr = item % pairs;
         const int a0 = 2 * pr, a1 = 2 * pr + 1;
         const bool has1 = a1 < R;
@@ -140,11 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
         __syncthreads();
         for (int hf = 0; hf < (has1 ? 2 : 1); ++hf) {
             const size_t row = (size_t)bh * R + (hf ? a1 : a0);
-            const int n8 = p.cnt[row], n4 = p.cnt[(size_t)BH * R + row];
+            const int n8 = p.cnt[row], n4 = p.cnt[BHR + row];
             const uint16_t* L0 = p.kidx + row * R;
             for (int i = tid; i < n8 + n4; i += kThreads) {
                 const int kb = L0[i];
-                if (kb >= R) { atomicOr(p.status, DA2_DEV_BADINDEX); continue; }
+                if (kb >= R) {
+                    atomicOr(p.status, DA2_DEV_BADINDEX);
+                    continue;
+                }
                 const int ph = i < n8 ? 0 : 1;
                 atomicOr(&bitmap[(ph * 2 + hf) * nwords + (kb >> 5)], 1u << (kb & 31));
             }
@@ -170,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
                         const int bit = __ffs(u) - 1;
                         u &= u - 1;
                         const int mask = ((m0 >> bit) & 1) | (((m1 >> bit) & 1) << 1);
-                        list[pos++] = Entry::make(w * 32 + bit, ph, mask);
+                        list[pos++] = make_entry(w * 32 + bit, ph, mask);
                     }
                     base += __shfl_sync(0xffffffffu, incl, 31);
                 }
@@ -197,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
                     const uint32_t g = gstep + j, st = g % kStages;
                     if (!mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status)) break;
                     const uint32_t e = list[j];
-                    const int kb = e & 0xFFFF, ph = (e >> 16) & 1;
+                    const int kb = e & 0xFFF, ph = (e >> 12) & 1;
                     const size_t tk = (size_t)bh * R + kb;
                     uint8_t* sb = smem + L::stage + st * L::stage_bytes;
                     if (ph == 0) {
@@ -228,15 +252,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
                     const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
                     if (!mbar_wait(&bar_p[pb], (g >> 1) & 1, abort_v, p.status)) return false;
                     tc_fence_after();
-                    const uint32_t e = list[i];
-                    const int ph = (e >> 16) & 1;
+                    const int ph = (list[i] >> 12) & 1;
                     uint8_t* sb = smem + L::stage + st * L::stage_bytes;
                     uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
                     if (ph == 0) {
 #pragma unroll
                         for (int kk = 0; kk < 2; ++kk)
-                            mma_f8(tmem + kColO, sdesc(pbuf + 256 * kk, 128, 512), sdesc(sb + L::v_off + 256 * kk, 128, 512),
-                                   idesc_f8(128, D), (i > 0 || kk > 0) ? 1u : 0u);
+                            mma_f8(tmem + kColO, sdesc(pbuf + 256 * kk, 128, 512),
+                                   sdesc(sb + L::v_off + 256 * kk, 128, 512), idesc_f8(128, D),
+                                   (i > 0 || kk > 0) ? 1u : 0u);
                     } else {
                         tc_cp_32x128_x4(tmem + kColSfp + 4 * pb, sdesc(pbuf + 128 * 64, 128, 128));
                         tc_cp_32x128_x4(tmem + kColSfv + 4 * pb, sdesc(sb + L::vsf_off, 128, 128));
@@ -248,146 +272,189 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
                     return true;
                 };
                 for (int j = 0; j < n_ent && ok; ++j) {
-                    const uint32_t g = gstep + j, st = g % kStages, sbuf = g & 1;
-                    if (!mbar_wait(&bar_full[st], (g / kStages) & 1, abort_v, p.status)) { ok = false; break; }
+                    const uint32_t g = gstep + j, st = g % kStages;
+                    if (!mbar_wait(&bar_full[st], (g / kStages) & 1, abort_v, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    // the S buffer is free once every softmax thread has read step g-1
+                    if (g > 0 && !mbar_wait(&bar_sfree, (g - 1) & 1, abort_v, p.status)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t e = list[j];
-                    const int ph = (e >> 16) & 1;
+                    const int ph = (list[j] >> 12) & 1;
                     uint8_t* sb = smem + L::stage + st * L::stage_bytes;
-                    const uint32_t sd = tmem + kColS + 64 * sbuf;
+                    const uint32_t sd = tmem + kColS;
                     if (ph == 0) {
 #pragma unroll
                         for (int kk = 0; kk < D / 32; ++kk)
-                            mma_f8(sd, sdesc(smem + L::q8 + 256 * kk, 128, 8 * D), sdesc(sb + L::k_off + 256 * kk, 128, 8 * D),
-                                   idesc_f8(128, 64), kk > 0 ? 1u : 0u);
+                            mma_f8(sd, sdesc(smem + L::q8 + 256 * kk, 128, 8 * D),
+                                   sdesc(sb + L::k_off + 256 * kk, 128, 8 * D), idesc_f8(128, 64), kk > 0 ? 1u : 0u);
                     } else {
-                        tc_cp_32x128_x4(tmem + kColSfk + 4 * sbuf, sdesc(sb + L::ksf_off, 128, 128));
+                        tc_cp_32x128_x4(tmem + kColSfk, sdesc(sb + L::ksf_off, 128, 128));
 #pragma unroll
                         for (int kk = 0; kk < D / 64; ++kk)
-                            mma_f4(sd, sdesc(smem + L::q4 + 256 * kk, 128, 4 * D), sdesc(sb + L::k_off + 256 * kk, 128, 4 * D),
-                                   idesc_f4(128, 64), tmem + kColSfq + 4 * kk, tmem + kColSfk + 4 * sbuf + 2 * kk,
-                                   kk > 0 ? 1u : 0u);
+                            mma_f4(sd, sdesc(smem + L::q4 + 256 * kk, 128, 4 * D),
+                                   sdesc(sb + L::k_off + 256 * kk, 128, 4 * D), idesc_f4(128, 64),
+                                   tmem + kColSfq + 4 * kk, tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
                     }
-                    tc_commit(&bar_s[sbuf]);
+                    tc_commit(&bar_s);
                     mma_issued = true;
-                    if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+                    if (j > 0 && !issue_pv(j - 1)) {
+                        ok = false;
+                        break;
+                    }
                 }
                 if (ok && n_ent > 0) ok = issue_pv(n_ent - 1);
+                // S buffer of the last step must be released before the next item's S
+                if (ok && n_ent > 0) mbar_wait(&bar_sfree, (gstep + n_ent - 1) & 1, abort_v, p.status);
             }
         } else {
             // ================================================== softmax
-            const int r = tid;            // tile row
-            const int hf = r >> 6;        // which query block of the pair
+            const int r = tid;      // tile row
+            const int hf = r >> 6;  // which query block of the pair
             const int a = hf ? a1 : a0;
             const bool qvalid = hf == 0 || has1;
             const size_t ta = (size_t)bh * R + (qvalid ? a : a0);
             const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-            const float rd = D == 64 ? 0.125f : 0.0883883461356163025f;  // 1/sqrt(D)
-            const float kLog2e = 1.4426950408889634f;
+            const float rdl2e = (D == 64 ? 0.125f : 0.0883883461356163025f) * 1.4426950408889634f;
             // Q scale factors of this row into the copy atoms (one per 64 channels)
             {
                 uint8_t* atom = smem + L::sfq;
                 const uint8_t* src = p.sfq + ta * (64 * (D / 16)) + (r & 63) * (D / 16);
                 for (int ch = 0; ch < D / 64; ++ch) {
-                    uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * ch) : 0u;
+                    const uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * ch) : 0u;
                     *reinterpret_cast<uint32_t*>(atom + 512 * ch + 16 * (r & 31) + 4 * (r >> 5)) = w;
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&bar_sfq);
             }
-            const float sq8 = p.scale[ta], gq4 = p.scale[(size_t)3 * BH * R + ta];
-            const float vm8 = p.vmax[bh], vm4 = p.vmax[BH + bh];
-            const float sig8 = __fdiv_rn(vm8, 448.0f), sig4 = __fdiv_rn(vm4, 2688.0f);
+            const float sq8 = p.scale[ta], gq4 = p.scale[3 * BHR + ta];
+            const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
+            const float switch_f = sig4 > 0.0f ? __fdiv_rn(sig8, sig4) : 1.0f;
+            auto load_meta = [&](int j) -> StepMeta {
+                StepMeta mt;
+                const uint32_t e = list[j];
+                const int kb = e & 0xFFF, ph = (e >> 12) & 1;
+                const size_t tk = (size_t)bh * R + kb;
+                mt.nk = p.n_a[kb];
+                mt.ck = p.scale[(ph ? 4 : 1) * BHR + tk];
+                const float vs = p.scale[(ph ? 5 : 2) * BHR + tk];
+                const float sg = ph ? sig4 : sig8;
+                mt.ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
+                return mt;
+            };
             float m = -INFINITY, l = 0.0f;
             bool ok = true;
+            StepMeta meta = n_ent > 0 ? load_meta(0) : StepMeta{0, 0.0f, 0.0f};
             for (int j = 0; j < n_ent && ok; ++j) {
-                const uint32_t g = gstep + j, sbuf = g & 1, pb = g & 1;
+                const uint32_t g = gstep + j, pb = g & 1;
                 const uint32_t e = list[j];
-                const int kb = e & 0xFFFF, ph = (e >> 16) & 1;
-                const bool active = (e >> (17 + hf)) & 1;
-                const size_t tk = (size_t)bh * R + kb;
-                const int nk = p.n_a[kb];
-                bool waited = mbar_wait(&bar_s[sbuf], (g >> 1) & 1, abort_v, p.status);
+                const int ph = (e >> 12) & 1;
+                const bool active = (e >> (13 + hf)) & 1;
+                bool waited = mbar_wait(&bar_s, g & 1, abort_v, p.status);
                 // P buffer pb was last read by the PV of step g-2
                 if (waited && g >= 2) waited = mbar_wait(&bar_pv[pb], ((g - 2) >> 1) & 1, abort_v, p.status);
-                if (!__all_sync(0xffffffffu, waited)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, waited)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
+                uint32_t s[64];
+                if (active) {
+                    tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+                    tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+                    tc_wait_ld();
+                }
+                tc_fence_before();
+                mbar_arrive(&bar_sfree);
+                const StepMeta mt = meta;
+                if (j + 1 < n_ent) meta = load_meta(j + 1);  // prefetch the next step's scalars
                 uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
                 float corr = 1.0f;
                 bool resc = false;
                 if (active) {
-                    uint32_t s[64];
-                    tmem_ld32(lane_base + kColS + 64 * sbuf, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-                    tmem_ld32(lane_base + kColS + 64 * sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-                    tc_wait_ld();
-                    const float cs = ph == 0 ? sq8 * p.scale[(size_t)BH * R + tk] : gq4 * p.scale[(size_t)4 * BH * R + tk];
-                    const float c2 = cs * rd * kLog2e;
-                    float mx = -INFINITY;
+                    // v = s * c (log2 units); the winning key gets v - m = 0
+                    // exactly, hence p = 1 exactly, as in the definition: the
+                    // product p * ratio then meets the same e4m3 / e2m1
+                    // rounding ties as p = e^(s - m) computed exactly.
+                    const float c2 = ((ph ? gq4 : sq8) * mt.ck) * rdl2e;
+                    const uint64_t c22 = pack2(c2, c2);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const float v = __uint_as_float(s[c]) * c2;
-                        s[c] = __float_as_uint(c < nk ? v : -INFINITY);
-                        mx = fmaxf(mx, __uint_as_float(s[c]));
+                    for (int c = 0; c < 64; c += 2) {
+                        const uint64_t v = mul2(pack2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c22);
+                        s[c] = __float_as_uint(lo2(v));
+                        s[c + 1] = __float_as_uint(hi2(v));
                     }
-                    const float mn = fmaxf(m, mx);
+                    if (mt.nk < 64) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (c >= mt.nk) s[c] = __float_as_uint(-INFINITY);
+                    }
+                    const float mn = fmaxf(m, rowmax64(s));
                     if (m != -INFINITY && mn > m) {
-                        corr = ex2(m - mn);
+                        corr = ex2f(m - mn);
                         resc = true;
                     }
-                    float sum = 0.0f;
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const float pv = ex2(__uint_as_float(s[c]) - mn);
-                        s[c] = __float_as_uint(pv);
-                        sum += pv;
-                    }
-                    l = l * corr + sum;
                     m = mn;
+                    const uint64_t nm2 = pack2(-mn, -mn);
+                    const uint64_t rt2 = pack2(mt.ratio, mt.ratio);
+                    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const uint64_t t = add2(pack2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), nm2);
+                        const uint64_t pp = pack2(ex2f(lo2(t)), ex2f(hi2(t)));
+                        acc[(c >> 1) & 3] = add2(acc[(c >> 1) & 3], pp);
+                        const uint64_t x = mul2(pp, rt2);  // p * ratio
+                        s[c] = __float_as_uint(lo2(x));
+                        s[c + 1] = __float_as_uint(hi2(x));
+                    }
+                    const uint64_t a2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+                    l = l * corr + (lo2(a2) + hi2(a2));
                     if (ph == 0) {
-                        const float ratio = sig8 > 0.0f ? __fdiv_rn(p.scale[(size_t)2 * BH * R + tk], sig8) : 0.0f;
 #pragma unroll
                         for (int ch = 0; ch < 4; ++ch) {
                             uint32_t w[4];
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
                                 const int c = ch * 16 + q * 4;
-                                const uint16_t lo = cvt_e4m3x2(__fmul_rn(__uint_as_float(s[c]), ratio),
-                                                               __fmul_rn(__uint_as_float(s[c + 1]), ratio));
-                                const uint16_t hi = cvt_e4m3x2(__fmul_rn(__uint_as_float(s[c + 2]), ratio),
-                                                               __fmul_rn(__uint_as_float(s[c + 3]), ratio));
-                                w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+                                const uint32_t lo = cvt_e4m3x2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                                const uint32_t hi = cvt_e4m3x2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+                                w[q] = lo | (hi << 16);
                             }
                             *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     } else {
-                        const float ratio = sig4 > 0.0f ? __fdiv_rn(p.scale[(size_t)5 * BH * R + tk], sig4) : 0.0f;
                         uint32_t sfw = 0;
 #pragma unroll
                         for (int gi = 0; gi < 4; ++gi) {
-                            float y[16], ym = 0.0f;
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) {
-                                y[q] = __fmul_rn(__uint_as_float(s[gi * 16 + q]), ratio);
-                                ym = fmaxf(ym, y[q]);
-                            }
-                            const uint8_t sf = (uint8_t)(cvt_e4m3x2(__fdiv_rn(ym, 6.0f), 0.0f) & 0xFF);
-                            const float rc = sf ? __fdiv_rn(1.0f, e4m3_to_f32(sf)) : 0.0f;
+                            const uint32_t* y = &s[gi * 16];
+                            const float t0 = max3f(__uint_as_float(y[0]), __uint_as_float(y[1]), __uint_as_float(y[2]));
+                            const float t1 = max3f(__uint_as_float(y[3]), __uint_as_float(y[4]), __uint_as_float(y[5]));
+                            const float t2 = max3f(__uint_as_float(y[6]), __uint_as_float(y[7]), __uint_as_float(y[8]));
+                            const float t3 = max3f(__uint_as_float(y[9]), __uint_as_float(y[10]), __uint_as_float(y[11]));
+                            const float t4 = max3f(__uint_as_float(y[12]), __uint_as_float(y[13]), __uint_as_float(y[14]));
+                            const float ym = max3f(max3f(t0, t1, t2), max3f(t3, t4, __uint_as_float(y[15])), 0.0f);
+                            const uint32_t sf = cvt_e4m3x2(__fdiv_rn(ym, 6.0f), 0.0f) & 0xFFu;
+                            const float rc = sf ? __frcp_rn(e4m3_to_f32((uint8_t)sf)) : 0.0f;
+                            const uint64_t rc2 = pack2(rc, rc);
                             uint32_t w[2];
 #pragma unroll
                             for (int hw = 0; hw < 2; ++hw) {
-                                uint32_t acc = 0;
+                                uint32_t accb = 0;
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) {
                                     const int c = hw * 8 + 2 * q;
-                                    const uint32_t byte = cvt_e2m1x2(__fmul_rn(y[c], rc), __fmul_rn(y[c + 1], rc));
-                                    acc |= byte << (8 * q);
+                                    const uint64_t yy = mul2(pack2(__uint_as_float(y[c]), __uint_as_float(y[c + 1])), rc2);
+                                    accb |= (uint32_t)cvt_e2m1x2(lo2(yy), hi2(yy)) << (8 * q);
                                 }
-                                w[hw] = sf ? acc : 0u;
+                                w[hw] = sf ? accb : 0u;
                             }
                             // 16 keys = 8 bytes: half of a 16-byte chunk
                             *reinterpret_cast<uint2*>(pbuf + kmajor_off(r, gi >> 1, 32) + 8 * (gi & 1)) =
                                 make_uint2(w[0], w[1]);
-                            sfw |= (uint32_t)sf << (8 * gi);
+                            sfw |= sf << (8 * gi);
                         }
                         *reinterpret_cast<uint32_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5)) = sfw;
                     }
@@ -407,23 +474,26 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
                 // O rescale: when the row max grew, and for every row at the
                 // switch from the 8-bit to the 4-bit phase (units sigma8 -> sigma4).
                 const bool sw = (j == n8e) && (j > 0);
-                float f = corr;
-                if (sw) f *= (sig4 > 0.0f ? __fdiv_rn(sig8, sig4) : 1.0f);
+                const float f = sw ? corr * switch_f : corr;
                 const bool need = (resc || sw) && j > 0;
                 if (__any_sync(0xffffffffu, need)) {
                     // O must hold the PV of step g-1 first
-                    const bool waited = mbar_wait(&bar_pv[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_v, p.status);
-                    if (!__all_sync(0xffffffffu, waited)) ok = false;
+                    const bool w2 = mbar_wait(&bar_pv[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_v, p.status);
+                    if (!__all_sync(0xffffffffu, w2)) ok = false;
                     if (ok) {
                         tc_fence_after();
-                        const float fm = need ? f : 1.0f;
-#pragma unroll
+                        const uint64_t f2 = need ? pack2(f, f) : pack2(1.0f, 1.0f);
+#pragma unroll 1
                         for (int c0 = 0; c0 < D; c0 += 32) {
                             uint32_t o[32];
                             tmem_ld32(lane_base + kColO + c0, o);
                             tc_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fm);
+                            for (int c = 0; c < 32; c += 2) {
+                                const uint64_t v = mul2(pack2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), f2);
+                                o[c] = __float_as_uint(lo2(v));
+                                o[c + 1] = __float_as_uint(hi2(v));
+                            }
                             tmem_st32(lane_base + kColO + c0, o);
                         }
                         tc_wait_st();
@@ -452,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
                 const int t = p.slot_token[a * 64 + qrow];
                 dst += (size_t)(bh / p.H) * p.o0 + (size_t)(bh % p.H) * p.o1 + (size_t)t * p.o2;
             }
-#pragma unroll
+#pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
                 if (have_o) {
@@ -478,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
             }
         }
         gstep += n_ent;
+        ++nitem;
     }
 
     // ---- teardown: drain outstanding async work, then free tensor memory
@@ -505,12 +576,13 @@ __global__ void __launch_bounds__(kThreads, 1) attention_kernel(AttnArgs p) {
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// At least 120 KB so that a single CTA fits on an SM: each CTA holds all 512
-// tensor-memory columns for its lifetime.
+// Two CTAs per SM: each needs at most ~113 KB of shared memory and at least
+// 80 KB, so that a third CTA never shares the SM (each CTA holds 256 of the
+// 512 tensor-memory columns for its lifetime).
 template <int D>
 size_t attention_smem_bytes(int R) {
-    const size_t need = Smem<D>::list + (size_t)2 * R * sizeof(uint32_t);
-    return need > 120 * 1024 ? need : 120 * 1024;
+    const size_t need = Smem<D>::list + (size_t)2 * R * sizeof(uint16_t);
+    return need > 80 * 1024 ? need : 80 * 1024;
 }
 
 }  // namespace
@@ -518,8 +590,9 @@ size_t attention_smem_bytes(int R) {
 cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream) {
     const int items = p.B * p.H * ((p.R + 1) / 2);
     if (items == 0) return cudaSuccess;
-    const int grid = items < p.num_sms ? items : p.num_sms;
-    cudaError_t e;
+    const int grid = items < 2 * p.num_sms ? items : 2 * p.num_sms;
+    cudaError_t e = cudaMemsetAsync(p.work_counter, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return e;
     if (p.d == 64) {
         const size_t smem = attention_smem_bytes<64>(p.R);
         e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

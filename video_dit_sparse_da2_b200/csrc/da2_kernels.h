@@ -64,6 +64,7 @@ struct AttnArgs {
     __nv_bfloat16* out;
     long long o0, o1, o2;  // element strides of the output
     unsigned* status;
+    int* work_counter;  // item counter of the persistent CTAs (zeroed per launch)
     int num_sms;
 };
 cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream);
