@@ -11,9 +11,12 @@
 // block kept that key block at that precision, so every row sees exactly its
 // own list in the order of the method.
 //
-// Roles (192 threads; two persistent CTAs per SM, each holding 256 of the
+// Roles (320 threads; two persistent CTAs per SM, each holding 256 of the
 // 512 tensor-memory columns; items fetched from a global counter):
-//   warps 0-3  softmax: thread r owns row r of the tile.  Reads S from tensor
+//   warps 0-7  softmax: two threads per row of the tile, each owning 32 of the
+//              64 key columns of a step (warp w reads tensor-memory lanes
+//              32*(w%4).. and columns 32*(w/4)..; the pair exchanges its
+//              partial row max through shared memory).  Reads S from tensor
 //              memory (then releases the S buffer at once), keeps the row max
 //              m and the unquantized denominator l (App. B.3), quantizes the
 //              weights into shared memory -- FP8: e4m3 of p times the value
@@ -24,10 +27,10 @@
 //              (sigma8 -> sigma4, the change of units of Eq. 8), and in the
 //              epilogue divides by l, converts to bf16 and stores the row at
 //              its original token position.
-//   warp 4     MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
+//   warp 8     MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
 //              kind::mxf4nvf4 block16) into the S buffer, O += P V into the
 //              single O accumulator.
-//   warp 5     loader (one thread): bulk async copies of the K / V tiles
+//   warp 9     loader (one thread): bulk async copies of the K / V tiles
 //              (pre-tiled by the preparation kernel) into a 3-stage ring.
 // Every mbarrier wait is bounded; a stuck wait sets the status word, all
 // roles drain their own outstanding work and the CTA frees tensor memory
@@ -40,8 +43,9 @@ namespace da2 {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kMmaWarp = 8, kLoadWarp = 9;
 constexpr uint32_t kTmemCols = 256;
 // tensor-memory column map (per CTA)
 constexpr uint32_t kColO = 0;      // O accumulator, D columns
@@ -72,7 +76,9 @@ struct Smem {
     static constexpr uint32_t p = stage + kStages * stage_bytes;  // 2 x (128 x 64 + 512)
     static constexpr uint32_t p_bytes = 128 * 64 + 512;
     static constexpr uint32_t bitmap = p + 2 * p_bytes;        // 4 x 128 words
-    static constexpr uint32_t list = bitmap + 4 * 128 * 4;     // 2R entries of 16 bits
+    static constexpr uint32_t xmax = bitmap + 4 * 128 * 4;     // [2 steps][2 halves][128 rows] floats
+    static constexpr uint32_t rcp = xmax + 2 * 2 * 128 * 4;    // 128 floats: 1/value of each ue4m3 code
+    static constexpr uint32_t list = rcp + 128 * 4;            // 2R entries of 16 bits
 };
 
 // Per-step scalars of a row: key-block size, score scale, value-scale ratio.
@@ -96,12 +102,30 @@ __device__ __forceinline__ float rowmax64(const uint32_t (&s)[64]) {
     return max3f(v0, v1, fmaxf(u[6], u[7]));
 }
 
+__device__ __forceinline__ float rowmax32(const uint32_t (&s)[32]) {
+    float t[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i)
+        t[i] = max3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]), __uint_as_float(s[3 * i + 2]));
+    t[10] = fmaxf(__uint_as_float(s[30]), __uint_as_float(s[31]));
+    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]), u2 = max3f(t[6], t[7], t[8]);
+    return max3f(max3f(u0, u1, u2), t[9], t[10]);
+}
+
+// x / 6 correctly rounded (q = x * RN(1/6), one fma residual correction).
+__device__ __forceinline__ float div6(float x) {
+    const float c = 0.16666667163372039794921875f;
+    const float q = x * c;
+    const float r = fmaf(-q, 6.0f, x);
+    return fmaf(r, c, q);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
     using L = Smem<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
-        bar_pv[2], bar_drain;
+        bar_pv[2], bar_x[4], bar_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh, item_sh;
     __shared__ int n_ent_sh[2];
@@ -129,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             mbar_init(&bar_p[s], kSoftmaxThreads);
             mbar_init(&bar_pv[s], 1);
         }
+        for (int s = 0; s < 4; ++s) mbar_init(&bar_x[s], 64);  // the two warps of a row quarter
         mbar_init(&bar_drain, 1);
         abort_sh = 0;
         fence_mbar_init();
@@ -136,6 +161,10 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
     if (warp == 0) {
         tmem_alloc(&tmem_base_sh, kTmemCols);
         tmem_relinquish();
+    }
+    {
+        float* rcp = reinterpret_cast<float*>(smem + L::rcp);
+        for (int c = tid; c < 128; c += kThreads) rcp[c] = c ? __frcp_rn(e4m3_to_f32((uint8_t)c)) : 0.0f;
     }
     tc_fence_before();
     __syncthreads();
@@ -145,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
     uint32_t gstep = 0;         // steps processed by this CTA before the current item
     uint32_t nitem = 0;         // items processed by this CTA
     uint32_t loads_issued = 0;  // loader: stage fills issued (for the final drain)
+    uint32_t nx = 0;            // softmax: exchanges with the partner warp so far
     bool mma_issued = false;
 
     for (;;) {
@@ -205,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
         __syncthreads();
         const int n8e = n_ent_sh[0], n_ent = n_ent_sh[0] + n_ent_sh[1];
 
-        if (warp == 5) {
+        if (warp == kLoadWarp) {
             // ================================================== loader
             if (lane == 0) {
                 const size_t t0 = (size_t)bh * R + a0;
@@ -238,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     ++loads_issued;
                 }
             }
-        } else if (warp == 4) {
+        } else if (warp == kMmaWarp) {
             // ================================================== MMA issue
             if (lane == 0) {
                 bool ok = mbar_wait(&bar_q, nitem & 1, abort_v, p.status);
@@ -312,24 +342,25 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             }
         } else {
             // ================================================== softmax
-            const int r = tid;      // tile row
-            const int hf = r >> 6;  // which query block of the pair
+            const int quarter = warp & 3, hh = warp >> 2;  // lane quarter, column half
+            const int r = 32 * quarter + lane;              // tile row
+            const int hf = r >> 6;                          // which query block of the pair
             const int a = hf ? a1 : a0;
             const bool qvalid = hf == 0 || has1;
             const size_t ta = (size_t)bh * R + (qvalid ? a : a0);
-            const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
             const float rdl2e = (D == 64 ? 0.125f : 0.0883883461356163025f) * 1.4426950408889634f;
+            float* xmax = reinterpret_cast<float*>(smem + L::xmax);
+            const float* rcp_tab = reinterpret_cast<const float*>(smem + L::rcp);
             // Q scale factors of this row into the copy atoms (one per 64 channels)
-            {
+            if (hh < D / 64) {
                 uint8_t* atom = smem + L::sfq;
                 const uint8_t* src = p.sfq + ta * (64 * (D / 16)) + (r & 63) * (D / 16);
-                for (int ch = 0; ch < D / 64; ++ch) {
-                    const uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * ch) : 0u;
-                    *reinterpret_cast<uint32_t*>(atom + 512 * ch + 16 * (r & 31) + 4 * (r >> 5)) = w;
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&bar_sfq);
+                const uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * hh) : 0u;
+                *reinterpret_cast<uint32_t*>(atom + 512 * hh + 16 * (r & 31) + 4 * (r >> 5)) = w;
             }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar_sfq);
             const float sq8 = p.scale[ta], gq4 = p.scale[3 * BHR + ta];
             const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
             const float switch_f = sig4 > 0.0f ? __fdiv_rn(sig8, sig4) : 1.0f;
@@ -345,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 mt.ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
                 return mt;
             };
-            float m = -INFINITY, l = 0.0f;
+            float m = -INFINITY, l = 0.0f;  // l: this thread's half of the denominator
             bool ok = true;
             StepMeta meta = n_ent > 0 ? load_meta(0) : StepMeta{0, 0.0f, 0.0f};
             for (int j = 0; j < n_ent && ok; ++j) {
@@ -361,10 +392,9 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     break;
                 }
                 tc_fence_after();
-                uint32_t s[64];
+                uint32_t s[32];
                 if (active) {
-                    tmem_ld32(lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-                    tmem_ld32(lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+                    tmem_ld32(lane_base + kColS + 32 * hh, s);
                     tc_wait_ld();
                 }
                 tc_fence_before();
@@ -382,17 +412,35 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     const float c2 = ((ph ? gq4 : sq8) * mt.ck) * rdl2e;
                     const uint64_t c22 = pack2(c2, c2);
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
+                    for (int c = 0; c < 32; c += 2) {
                         const uint64_t v = mul2(pack2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c22);
                         s[c] = __float_as_uint(lo2(v));
                         s[c + 1] = __float_as_uint(hi2(v));
                     }
-                    if (mt.nk < 64) {
+                    const int nk = mt.nk - 32 * hh;  // valid keys among this thread's columns
+                    if (nk < 32) {
+                        if (nk >= 16) {
 #pragma unroll
-                        for (int c = 0; c < 64; ++c)
-                            if (c >= mt.nk) s[c] = __float_as_uint(-INFINITY);
+                            for (int c = 16; c < 32; ++c)
+                                if (c >= nk) s[c] = __float_as_uint(-INFINITY);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (c >= nk) s[c] = __float_as_uint(-INFINITY);
+                        }
                     }
-                    const float mn = fmaxf(m, rowmax64(s));
+                    // row max over both halves: exchange with the partner warp
+                    // (two slots alternating by exchange parity)
+                    float* xm = xmax + (nx & 1) * 256;
+                    xm[hh * 128 + r] = rowmax32(s);
+                    mbar_arrive(&bar_x[quarter]);
+                    const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
+                    ++nx;
+                    if (!__all_sync(0xffffffffu, xw)) {
+                        ok = false;
+                        break;
+                    }
+                    const float mn = fmaxf(m, fmaxf(xm[r], xm[128 + r]));
                     if (m != -INFINITY && mn > m) {
                         corr = ex2f(m - mn);
                         resc = true;
@@ -400,21 +448,21 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     m = mn;
                     const uint64_t nm2 = pack2(-mn, -mn);
                     const uint64_t rt2 = pack2(mt.ratio, mt.ratio);
-                    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+                    uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
+                    for (int c = 0; c < 32; c += 2) {
                         const uint64_t t = add2(pack2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), nm2);
                         const uint64_t pp = pack2(ex2f(lo2(t)), ex2f(hi2(t)));
-                        acc[(c >> 1) & 3] = add2(acc[(c >> 1) & 3], pp);
+                        acc[(c >> 1) & 1] = add2(acc[(c >> 1) & 1], pp);
                         const uint64_t x = mul2(pp, rt2);  // p * ratio
                         s[c] = __float_as_uint(lo2(x));
                         s[c + 1] = __float_as_uint(hi2(x));
                     }
-                    const uint64_t a2 = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+                    const uint64_t a2 = add2(acc[0], acc[1]);
                     l = l * corr + (lo2(a2) + hi2(a2));
                     if (ph == 0) {
 #pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) {
+                        for (int ch = 0; ch < 2; ++ch) {
                             uint32_t w[4];
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
@@ -423,12 +471,13 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                                 const uint32_t hi = cvt_e4m3x2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
                                 w[q] = lo | (hi << 16);
                             }
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 2 * hh + ch, 64)) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     } else {
-                        uint32_t sfw = 0;
+                        uint32_t sfw = 0, wq[4];
 #pragma unroll
-                        for (int gi = 0; gi < 4; ++gi) {
+                        for (int gi = 0; gi < 2; ++gi) {
                             const uint32_t* y = &s[gi * 16];
                             const float t0 = max3f(__uint_as_float(y[0]), __uint_as_float(y[1]), __uint_as_float(y[2]));
                             const float t1 = max3f(__uint_as_float(y[3]), __uint_as_float(y[4]), __uint_as_float(y[5]));
@@ -436,10 +485,9 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                             const float t3 = max3f(__uint_as_float(y[9]), __uint_as_float(y[10]), __uint_as_float(y[11]));
                             const float t4 = max3f(__uint_as_float(y[12]), __uint_as_float(y[13]), __uint_as_float(y[14]));
                             const float ym = max3f(max3f(t0, t1, t2), max3f(t3, t4, __uint_as_float(y[15])), 0.0f);
-                            const uint32_t sf = cvt_e4m3x2(__fdiv_rn(ym, 6.0f), 0.0f) & 0xFFu;
-                            const float rc = sf ? __frcp_rn(e4m3_to_f32((uint8_t)sf)) : 0.0f;
+                            const uint32_t sf = cvt_e4m3x2(div6(ym), 0.0f) & 0x7Fu;
+                            const float rc = rcp_tab[sf];
                             const uint64_t rc2 = pack2(rc, rc);
-                            uint32_t w[2];
 #pragma unroll
                             for (int hw = 0; hw < 2; ++hw) {
                                 uint32_t accb = 0;
@@ -449,30 +497,29 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                                     const uint64_t yy = mul2(pack2(__uint_as_float(y[c]), __uint_as_float(y[c + 1])), rc2);
                                     accb |= (uint32_t)cvt_e2m1x2(lo2(yy), hi2(yy)) << (8 * q);
                                 }
-                                w[hw] = sf ? accb : 0u;
+                                wq[2 * gi + hw] = sf ? accb : 0u;
                             }
-                            // 16 keys = 8 bytes: half of a 16-byte chunk
-                            *reinterpret_cast<uint2*>(pbuf + kmajor_off(r, gi >> 1, 32) + 8 * (gi & 1)) =
-                                make_uint2(w[0], w[1]);
                             sfw |= sf << (8 * gi);
                         }
-                        *reinterpret_cast<uint32_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5)) = sfw;
+                        // 32 keys = one 16-byte chunk of the 32-byte row
+                        *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, hh, 32)) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                        *reinterpret_cast<uint16_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5) + 2 * hh) =
+                            (uint16_t)sfw;
                     }
                 } else {
                     // row not in this step: zero weights
                     if (ph == 0) {
 #pragma unroll
-                        for (int ch = 0; ch < 4; ++ch)
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) = make_uint4(0, 0, 0, 0);
-                    } else {
-#pragma unroll
                         for (int ch = 0; ch < 2; ++ch)
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 32)) = make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint32_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5)) = 0u;
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 2 * hh + ch, 64)) = make_uint4(0, 0, 0, 0);
+                    } else {
+                        *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, hh, 32)) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint16_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5) + 2 * hh) = 0;
                     }
                 }
-                // O rescale: when the row max grew, and for every row at the
-                // switch from the 8-bit to the 4-bit phase (units sigma8 -> sigma4).
+                // O rescale (this thread's half of the columns): when the row
+                // max grew, and for every row at the switch from the 8-bit to
+                // the 4-bit phase (units sigma8 -> sigma4).
                 const bool sw = (j == n8e) && (j > 0);
                 const float f = sw ? corr * switch_f : corr;
                 const bool need = (resc || sw) && j > 0;
@@ -484,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                         tc_fence_after();
                         const uint64_t f2 = need ? pack2(f, f) : pack2(1.0f, 1.0f);
 #pragma unroll 1
-                        for (int c0 = 0; c0 < D; c0 += 32) {
+                        for (int c0 = hh * (D / 2); c0 < (hh + 1) * (D / 2); c0 += 32) {
                             uint32_t o[32];
                             tmem_ld32(lane_base + kColO + c0, o);
                             tc_wait_ld();
@@ -503,8 +550,18 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 tc_fence_before();
                 mbar_arrive(&bar_p[pb]);
             }
-            // ---- epilogue
+            // ---- epilogue: both halves of the denominator, then this thread's columns
             ok = __all_sync(0xffffffffu, ok);
+            float lt = 0.0f;
+            {
+                float* xl = xmax + (nx & 1) * 256;
+                xl[hh * 128 + r] = l;
+                mbar_arrive(&bar_x[quarter]);
+                const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
+                ++nx;
+                if (!__all_sync(0xffffffffu, xw)) ok = false;
+                lt = xl[r] + xl[128 + r];
+            }
             float o_scale = 0.0f;
             const bool have = n_ent > 0 && ok;
             if (have) {
@@ -512,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 if (!mbar_wait(&bar_pv[g & 1], (g >> 1) & 1, abort_v, p.status)) ok = false;
                 tc_fence_after();
                 const float unit = n_ent > n8e ? sig4 : sig8;
-                o_scale = l > 0.0f ? __fdiv_rn(unit, l) : 0.0f;
+                o_scale = lt > 0.0f ? __fdiv_rn(unit, lt) : 0.0f;
             }
             const bool have_o = __all_sync(0xffffffffu, have && ok);
             const int qrow = r & 63;
@@ -523,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 dst += (size_t)(bh / p.H) * p.o0 + (size_t)(bh % p.H) * p.o1 + (size_t)t * p.o2;
             }
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = hh * (D / 2); c0 < (hh + 1) * (D / 2); c0 += 32) {
                 uint32_t o[32];
                 if (have_o) {
                     tmem_ld32(lane_base + kColO + c0, o);
@@ -532,19 +589,20 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
 #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = 0u;
                 }
-                if (!store) continue;
-                uint32_t packed[16];
+                if (store) {
+                    uint32_t packed[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float x0 = o_scale > 0.0f ? __uint_as_float(o[2 * c]) * o_scale : 0.0f;
-                    const float x1 = o_scale > 0.0f ? __uint_as_float(o[2 * c + 1]) * o_scale : 0.0f;
-                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
-                    packed[c] = *reinterpret_cast<const uint32_t*>(&b2);
+                    for (int c = 0; c < 16; ++c) {
+                        const float x0 = o_scale > 0.0f ? __uint_as_float(o[2 * c]) * o_scale : 0.0f;
+                        const float x1 = o_scale > 0.0f ? __uint_as_float(o[2 * c + 1]) * o_scale : 0.0f;
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                        packed[c] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        *reinterpret_cast<uint4*>(dst + c0 + 8 * v) =
+                            make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                 }
-#pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    *reinterpret_cast<uint4*>(dst + c0 + 8 * v) =
-                        make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
             }
         }
         gstep += n_ent;
@@ -553,21 +611,15 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
 
     // ---- teardown: drain outstanding async work, then free tensor memory
     __syncthreads();
-    if (warp == 4 && lane == 0 && mma_issued) {
+    if (warp == kMmaWarp && lane == 0 && mma_issued) {
         tc_commit(&bar_drain);
-        for (uint32_t i = 0; i < DA2_WAIT_LIMIT; ++i) {
-            if (mbar_try_wait(&bar_drain, 0)) break;
-            __nanosleep(128);
-        }
+        if (!mbar_wait_drain(&bar_drain, 0)) atomicOr(p.status, DA2_DEV_TIMEOUT);
     }
-    if (warp == 5 && lane == 0) {
+    if (warp == kLoadWarp && lane == 0) {
         // every issued stage fill must have landed before the CTA exits
         for (uint32_t k = 0; k < loads_issued && k < (uint32_t)kStages; ++k) {
             const uint32_t g = loads_issued - 1 - k, st = g % kStages;
-            for (uint32_t i = 0; i < DA2_WAIT_LIMIT; ++i) {
-                if (mbar_try_wait(&bar_full[st], (g / kStages) & 1)) break;
-                __nanosleep(128);
-            }
+            if (!mbar_wait_drain(&bar_full[st], (g / kStages) & 1)) atomicOr(p.status, DA2_DEV_TIMEOUT);
         }
     }
     tc_fence_before();

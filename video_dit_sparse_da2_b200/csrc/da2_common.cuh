@@ -13,9 +13,12 @@
 #define DA2_DEV_TIMEOUT 1u
 #define DA2_DEV_BADINDEX 2u
 
-// Polls of an mbarrier before a wait is declared stuck (with back-off this is
-// several seconds, far beyond any legitimate wait in these kernels).
-#define DA2_WAIT_LIMIT (1u << 24)
+// A device-side wait is declared stuck after this many nanoseconds (far
+// beyond any legitimate wait in these kernels).
+#define DA2_WAIT_NS 4000000000ull
+// Suspend-time hint of one mbarrier try_wait: the waiting thread sleeps in
+// hardware until the phase completes or this many nanoseconds pass.
+#define DA2_SUSPEND_NS 100000u
 
 namespace da2 {
 
@@ -49,19 +52,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that may suspend the thread for up to `ns` nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
 // Bounded wait: returns false (and sets *status) when the barrier does not
-// complete the given phase within DA2_WAIT_LIMIT polls, or when another warp
-// already gave up (*abort set).
+// complete the given phase within DA2_WAIT_NS, or when another warp already
+// gave up (*abort set).  The thread sleeps inside try_wait between checks.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned* status) {
-    for (uint32_t i = 0; i < DA2_WAIT_LIMIT; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, DA2_SUSPEND_NS)) return true;
         if (*abort) return false;
-        if (i > 64) __nanosleep(i > 4096 ? 256 : 32);
+        if (globaltimer_ns() - t0 > DA2_WAIT_NS) break;
     }
     *abort = 1;
     atomicOr(status, DA2_DEV_TIMEOUT);
     return false;
+}
+// Bounded wait without the abort short-cut (used to drain own async work).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, DA2_SUSPEND_NS)) return true;
+        if (globaltimer_ns() - t0 > DA2_WAIT_NS) return false;
+    }
 }
 
 // -------------------------------------------------------- bulk async copy
