@@ -167,6 +167,35 @@ int da2_prepare(da2_handle h, const void* q, const void* k, const void* v, const
 int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, const da2_plan_bufs* plan,
              void* stream);
 
+/* Size of the working memory da2_plan_static keeps inside the library:
+ * 32 MiB of device memory on every GPU where the library is used, held until
+ * the process exits. */
+#define DA2_PLAN_STATIC_BYTES (32u << 20)
+
+/* da2_plan for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a service of the library.  Some callers must not call
+ * cudaMalloc at the moment they route: code recording a CUDA graph by stream
+ * capture (allocation is not allowed while a capture is open), hosts that own
+ * all device memory through their own pools and forbid plugins to allocate,
+ * and latency-critical paths where cudaMalloc's implicit synchronization
+ * would stall other streams.  This entry point computes exactly what da2_plan
+ * computes (same kernels, same results) but takes no scratch buffer: its
+ * working memory is a fixed DA2_PLAN_STATIC_BYTES array inside the library.
+ * The caller still passes the prepared operands and the four outputs (prec,
+ * cnt, kidx, A, device, layouts as in da2_plan_bufs).
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture begins.
+ *   - Every call reuses the same array and clears what must start at zero;
+ *     two calls that overlap on the same GPU (different streams, threads or
+ *     handles) race on it: order them.
+ *   - Returns DA2_ERR_ARG, without enqueueing anything, when the shape needs
+ *     more working memory than DA2_PLAN_STATIC_BYTES (da2_sizes' plan_scratch
+ *     tells how much: about B*H*R*R*8 bytes plus 33 KB per head).  Other
+ *     errors as da2_plan. */
+int da2_plan_static(da2_handle h, const da2_prepared* prep, const da2_budget* budget, uint8_t* prec, int32_t* cnt,
+                    uint16_t* kidx, double* A, void* stream);
+
 /* Block-sparse mixed-precision attention (Sec. 3.3; App. B.3, C.1).  out:
  * bf16 (device), [B][H][N][d] with strides out_strides[] in elements
  * (out_strides[3] == 1); every token row is written (rows with no retained

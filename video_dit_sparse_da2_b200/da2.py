@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libda2.so")
 OK, ERR_ARG, ERR_ARCH, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
 
 # Every symbol include/da2.h declares.
-EXPORTS = ("da2_create", "da2_destroy", "da2_partition", "da2_sizes", "da2_tables", "da2_prepare", "da2_plan", "da2_attention",
+EXPORTS = ("da2_create", "da2_destroy", "da2_partition", "da2_sizes", "da2_tables", "da2_prepare", "da2_plan",
+           "da2_plan_static", "da2_attention",
            "da2_check_device_status", "da2_status_string", "da2_last_cuda_error")
 
 
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.da2_tables.argtypes = [P, P, P]
         L.da2_prepare.argtypes = [P, P, P, P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(PreparedPtrs), P]
         L.da2_plan.argtypes = [P, ctypes.POINTER(PreparedPtrs), ctypes.POINTER(Budget), ctypes.POINTER(PlanPtrs), P]
+        L.da2_plan_static.argtypes = [P, ctypes.POINTER(PreparedPtrs), ctypes.POINTER(Budget), P, P, P, P, P]
         L.da2_attention.argtypes = [P, ctypes.POINTER(PreparedPtrs), ctypes.POINTER(PlanPtrs), P,
                                     ctypes.POINTER(ctypes.c_int64), P]
         L.da2_check_device_status.argtypes = [P, P]
@@ -182,6 +184,21 @@ class DA2:
         b = Budget(int(bp8), int(bp4), float(lam))
         _check(lib().da2_plan(self.handle, ctypes.byref(prep.ptrs()), ctypes.byref(b), ctypes.byref(plan.ptrs()),
                               _stream_ptr(stream)), "da2_plan")
+
+    def plan_static(self, prep: Prepared, plan: Plan, bp8: int, bp4: int, lam: float = 0.2, stream=None):
+        """Routing without a caller scratch buffer (da2_plan_static): for callers
+        that cannot allocate device memory, e.g. while capturing a CUDA graph.
+        Writes plan.bufs' prec / cnt / kidx / A; plan.bufs["scratch"] is unused."""
+        need = int(self.sizes.plan_scratch)
+        limit = 32 << 20
+        if need > limit:
+            raise DA2Error(f"da2_plan_static: this shape needs {need} bytes of working memory, "
+                           f"more than the library's fixed {limit} bytes; use plan() with a scratch buffer")
+        b = Budget(int(bp8), int(bp4), float(lam))
+        bufs = plan.bufs
+        _check(lib().da2_plan_static(self.handle, ctypes.byref(prep.ptrs()), ctypes.byref(b), bufs["prec"].data_ptr(),
+                                     bufs["cnt"].data_ptr(), bufs["kidx"].data_ptr(), bufs["A"].data_ptr(),
+                                     _stream_ptr(stream)), "da2_plan_static")
 
     def attention(self, prep: Prepared, plan: Plan, out: torch.Tensor, stream=None):
         assert out.dtype == torch.bfloat16
