@@ -88,36 +88,74 @@ struct StepMeta {
     float ratio;  // V tile scale over the phase unit
 };
 
-__device__ __forceinline__ float rowmax64(const uint32_t (&s)[64]) {
-    float t[22];
-#pragma unroll
-    for (int i = 0; i < 21; ++i)
-        t[i] = max3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]), __uint_as_float(s[3 * i + 2]));
-    t[21] = __uint_as_float(s[63]);
-    float u[8];
-#pragma unroll
-    for (int i = 0; i < 7; ++i) u[i] = max3f(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
-    u[7] = t[21];
-    const float v0 = max3f(u[0], u[1], u[2]), v1 = max3f(u[3], u[4], u[5]);
-    return max3f(v0, v1, fmaxf(u[6], u[7]));
-}
-
-__device__ __forceinline__ float rowmax32(const uint32_t (&s)[32]) {
-    float t[11];
-#pragma unroll
-    for (int i = 0; i < 10; ++i)
-        t[i] = max3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]), __uint_as_float(s[3 * i + 2]));
-    t[10] = fmaxf(__uint_as_float(s[30]), __uint_as_float(s[31]));
-    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]), u2 = max3f(t[6], t[7], t[8]);
-    return max3f(max3f(u0, u1, u2), t[9], t[10]);
-}
-
 // x / 6 correctly rounded (q = x * RN(1/6), one fma residual correction).
 __device__ __forceinline__ float div6(float x) {
     const float c = 0.16666667163372039794921875f;
     const float q = x * c;
     const float r = fmaf(-q, 6.0f, x);
     return fmaf(r, c, q);
+}
+
+// 32 consecutive fp32 columns of this warp's tensor-memory lanes, as pairs;
+// load and wait in one asm statement (see tmem_ld32).
+__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr, float2 (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x),
+          "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y),
+          "=f"(v[7].x), "=f"(v[7].y), "=f"(v[8].x), "=f"(v[8].y), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[10].x),
+          "=f"(v[10].y), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[13].x),
+          "=f"(v[13].y), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[15].x), "=f"(v[15].y)
+        : "r"(taddr)
+        : "memory");
+}
+
+// Four fp32 -> four e4m3 bytes in one word (first value in the low byte).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float2 a, float2 b) {
+    uint32_t w;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return w;
+}
+
+// Eight fp32 -> eight e2m1 nibbles in one word (first value in the low nibble).
+__device__ __forceinline__ uint32_t pack_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+    return w;
+}
+
+__device__ __forceinline__ float rowmax32f2(const float2 (&v)[16]) {
+    float t[11];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        t[2 * i] = max3f(v[3 * i].x, v[3 * i].y, v[3 * i + 1].x);
+        t[2 * i + 1] = max3f(v[3 * i + 1].y, v[3 * i + 2].x, v[3 * i + 2].y);
+    }
+    t[10] = fmaxf(v[15].x, v[15].y);
+    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]), u2 = max3f(t[6], t[7], t[8]);
+    return max3f(max3f(u0, u1, u2), t[9], t[10]);
+}
+
+// Max of 16 consecutive values v[b..b+7] (pairs) and 0.
+__device__ __forceinline__ float groupmax16(const float2 (&v)[16], int b) {
+    const float t0 = max3f(v[b].x, v[b].y, v[b + 1].x), t1 = max3f(v[b + 1].y, v[b + 2].x, v[b + 2].y);
+    const float t2 = max3f(v[b + 3].x, v[b + 3].y, v[b + 4].x), t3 = max3f(v[b + 4].y, v[b + 5].x, v[b + 5].y);
+    const float t4 = max3f(v[b + 6].x, v[b + 6].y, v[b + 7].x);
+    return max3f(max3f(t0, t1, t2), max3f(t3, t4, v[b + 7].y), 0.0f);
 }
 
 template <int D>
@@ -392,10 +430,9 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     break;
                 }
                 tc_fence_after();
-                uint32_t s[32];
+                float2 v[16];
                 if (active) {
-                    tmem_ld32(lane_base + kColS + 32 * hh, s);
-                    tc_wait_ld();
+                    tmem_ld32x2(lane_base + kColS + 32 * hh, v);
                 }
                 tc_fence_before();
                 mbar_arrive(&bar_sfree);
@@ -410,29 +447,29 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     // product p * ratio then meets the same e4m3 / e2m1
                     // rounding ties as p = e^(s - m) computed exactly.
                     const float c2 = ((ph ? gq4 : sq8) * mt.ck) * rdl2e;
-                    const uint64_t c22 = pack2(c2, c2);
+                    const float2 c22 = make_float2(c2, c2);
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const uint64_t v = mul2(pack2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c22);
-                        s[c] = __float_as_uint(lo2(v));
-                        s[c + 1] = __float_as_uint(hi2(v));
-                    }
+                    for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], c22);
                     const int nk = mt.nk - 32 * hh;  // valid keys among this thread's columns
                     if (nk < 32) {
                         if (nk >= 16) {
 #pragma unroll
-                            for (int c = 16; c < 32; ++c)
-                                if (c >= nk) s[c] = __float_as_uint(-INFINITY);
+                            for (int i = 8; i < 16; ++i) {
+                                if (2 * i >= nk) v[i].x = -INFINITY;
+                                if (2 * i + 1 >= nk) v[i].y = -INFINITY;
+                            }
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                if (c >= nk) s[c] = __float_as_uint(-INFINITY);
+                            for (int i = 0; i < 16; ++i) {
+                                if (2 * i >= nk) v[i].x = -INFINITY;
+                                if (2 * i + 1 >= nk) v[i].y = -INFINITY;
+                            }
                         }
                     }
                     // row max over both halves: exchange with the partner warp
                     // (two slots alternating by exchange parity)
                     float* xm = xmax + (nx & 1) * 256;
-                    xm[hh * 128 + r] = rowmax32(s);
+                    xm[hh * 128 + r] = rowmax32f2(v);
                     mbar_arrive(&bar_x[quarter]);
                     const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
                     ++nx;
@@ -446,59 +483,43 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                         resc = true;
                     }
                     m = mn;
-                    const uint64_t nm2 = pack2(-mn, -mn);
-                    const uint64_t rt2 = pack2(mt.ratio, mt.ratio);
-                    uint64_t acc[2] = {0ull, 0ull};
+                    const float2 nm = make_float2(-mn, -mn);
+                    const float2 rt = make_float2(mt.ratio, mt.ratio);
+                    float2 acc0 = make_float2(0.0f, 0.0f), acc1 = acc0;
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const uint64_t t = add2(pack2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), nm2);
-                        const uint64_t pp = pack2(ex2f(lo2(t)), ex2f(hi2(t)));
-                        acc[(c >> 1) & 1] = add2(acc[(c >> 1) & 1], pp);
-                        const uint64_t x = mul2(pp, rt2);  // p * ratio
-                        s[c] = __float_as_uint(lo2(x));
-                        s[c + 1] = __float_as_uint(hi2(x));
+                    for (int i = 0; i < 16; i += 2) {
+                        const float2 t0 = __fadd2_rn(v[i], nm), t1 = __fadd2_rn(v[i + 1], nm);
+                        const float2 p0 = make_float2(ex2f(t0.x), ex2f(t0.y));
+                        const float2 p1 = make_float2(ex2f(t1.x), ex2f(t1.y));
+                        acc0 = __fadd2_rn(acc0, p0);
+                        acc1 = __fadd2_rn(acc1, p1);
+                        v[i] = __fmul2_rn(p0, rt);  // p * ratio
+                        v[i + 1] = __fmul2_rn(p1, rt);
                     }
-                    const uint64_t a2 = add2(acc[0], acc[1]);
-                    l = l * corr + (lo2(a2) + hi2(a2));
+                    const float2 a2 = __fadd2_rn(acc0, acc1);
+                    l = l * corr + (a2.x + a2.y);
                     if (ph == 0) {
 #pragma unroll
                         for (int ch = 0; ch < 2; ++ch) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const int c = ch * 16 + q * 4;
-                                const uint32_t lo = cvt_e4m3x2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-                                const uint32_t hi = cvt_e4m3x2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
-                                w[q] = lo | (hi << 16);
-                            }
+                            const int b = ch * 8;
                             *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 2 * hh + ch, 64)) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
+                                make_uint4(pack_e4m3x4(v[b], v[b + 1]), pack_e4m3x4(v[b + 2], v[b + 3]),
+                                           pack_e4m3x4(v[b + 4], v[b + 5]), pack_e4m3x4(v[b + 6], v[b + 7]));
                         }
                     } else {
                         uint32_t sfw = 0, wq[4];
 #pragma unroll
                         for (int gi = 0; gi < 2; ++gi) {
-                            const uint32_t* y = &s[gi * 16];
-                            const float t0 = max3f(__uint_as_float(y[0]), __uint_as_float(y[1]), __uint_as_float(y[2]));
-                            const float t1 = max3f(__uint_as_float(y[3]), __uint_as_float(y[4]), __uint_as_float(y[5]));
-                            const float t2 = max3f(__uint_as_float(y[6]), __uint_as_float(y[7]), __uint_as_float(y[8]));
-                            const float t3 = max3f(__uint_as_float(y[9]), __uint_as_float(y[10]), __uint_as_float(y[11]));
-                            const float t4 = max3f(__uint_as_float(y[12]), __uint_as_float(y[13]), __uint_as_float(y[14]));
-                            const float ym = max3f(max3f(t0, t1, t2), max3f(t3, t4, __uint_as_float(y[15])), 0.0f);
+                            const int b = gi * 8;
+                            const float ym = groupmax16(v, b);
                             const uint32_t sf = cvt_e4m3x2(div6(ym), 0.0f) & 0x7Fu;
                             const float rc = rcp_tab[sf];
-                            const uint64_t rc2 = pack2(rc, rc);
+                            const float2 rc2 = make_float2(rc, rc);
+                            float2 y[8];
 #pragma unroll
-                            for (int hw = 0; hw < 2; ++hw) {
-                                uint32_t accb = 0;
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const int c = hw * 8 + 2 * q;
-                                    const uint64_t yy = mul2(pack2(__uint_as_float(y[c]), __uint_as_float(y[c + 1])), rc2);
-                                    accb |= (uint32_t)cvt_e2m1x2(lo2(yy), hi2(yy)) << (8 * q);
-                                }
-                                wq[2 * gi + hw] = sf ? accb : 0u;
-                            }
+                            for (int i = 0; i < 8; ++i) y[i] = __fmul2_rn(v[b + i], rc2);
+                            wq[2 * gi] = sf ? pack_e2m1x8(y[0], y[1], y[2], y[3]) : 0u;
+                            wq[2 * gi + 1] = sf ? pack_e2m1x8(y[4], y[5], y[6], y[7]) : 0u;
                             sfw |= sf << (8 * gi);
                         }
                         // 32 keys = one 16-byte chunk of the 32-byte row
@@ -534,7 +555,6 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                         for (int c0 = hh * (D / 2); c0 < (hh + 1) * (D / 2); c0 += 32) {
                             uint32_t o[32];
                             tmem_ld32(lane_base + kColO + c0, o);
-                            tc_wait_ld();
 #pragma unroll
                             for (int c = 0; c < 32; c += 2) {
                                 const uint64_t v = mul2(pack2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), f2);
@@ -584,7 +604,6 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 uint32_t o[32];
                 if (have_o) {
                     tmem_ld32(lane_base + kColO + c0, o);
-                    tc_wait_ld();
                 } else {
 #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = 0u;
