@@ -11,26 +11,28 @@
 // block kept that key block at that precision, so every row sees exactly its
 // own list in the order of the method.
 //
-// Roles (320 threads; two persistent CTAs per SM, each holding 256 of the
-// 512 tensor-memory columns; items fetched from a global counter):
-//   warps 0-7  softmax: two threads per row of the tile, each owning 32 of the
-//              64 key columns of a step (warp w reads tensor-memory lanes
-//              32*(w%4).. and columns 32*(w/4)..; the pair exchanges its
-//              partial row max through shared memory).  Reads S from tensor
-//              memory (then releases the S buffer at once), keeps the row max
-//              m and the unquantized denominator l (App. B.3), quantizes the
-//              weights into shared memory -- FP8: e4m3 of p times the value
-//              tile scale over the phase unit; NVFP4: that product quantized
-//              per 16 keys with a ue4m3 scale -- with the same fp32 rounding
-//              steps as the definition (p of the winning key is exactly 1),
-//              rescales its row of O when m grows and once at the phase switch
-//              (sigma8 -> sigma4, the change of units of Eq. 8), and in the
-//              epilogue divides by l, converts to bf16 and stores the row at
-//              its original token position.
-//   warp 8     MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
+// Roles (192 threads with one softmax thread per row; two persistent CTAs per
+// SM, each holding 256 of the 512 tensor-memory columns; items fetched from a
+// global counter):
+//   warps 0-3  softmax: one thread per row of the tile (warp w reads
+//              tensor-memory lanes 32w..32w+31, all 64 key columns of a step).
+//              Reads S from tensor memory (then releases the S buffer at
+//              once), keeps the row max m and the unquantized denominator l
+//              (App. B.3), quantizes the weights into shared memory -- FP8:
+//              e4m3 of p times the value tile scale over the phase unit;
+//              NVFP4: that product quantized per 16 keys with a ue4m3 scale --
+//              with the same fp32 rounding steps as the definition (p of the
+//              winning key is exactly 1), rescales its row of O when m grows
+//              and once at the phase switch (sigma8 -> sigma4, the change of
+//              units of Eq. 8), and in the epilogue divides by l, converts to
+//              bf16 and stores the row at its original token position.  The
+//              template also builds a two-threads-per-row split (RT = 2: 8
+//              softmax warps, each owning 32 of the 64 columns, the pair
+//              exchanging its partial row max through shared memory).
+//   warp 4RT   MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
 //              kind::mxf4nvf4 block16) into the S buffer, O += P V into the
 //              single O accumulator.
-//   warp 9     loader (one thread): bulk async copies of the K / V tiles
+//   warp 4RT+1 loader (one thread): bulk async copies of the K / V tiles
 //              (pre-tiled by the preparation kernel) into a 3-stage ring.
 // Every mbarrier wait is bounded; a stuck wait sets the status word, all
 // roles drain their own outstanding work and the CTA frees tensor memory
@@ -43,9 +45,18 @@ namespace da2 {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
-constexpr int kSoftmaxThreads = 256;
-constexpr int kMmaWarp = 8, kLoadWarp = 9;
+// Softmax threads per row of the tile (1: each thread owns all 64 key columns
+// of a step; 2: two threads split them and exchange the partial row max).
+constexpr int kRowThreads = 1;
+
+template <int RT>
+struct Cfg {
+    static constexpr int kSoftThreads = 128 * RT;
+    static constexpr int kThreads = kSoftThreads + 64;
+    static constexpr int kMmaWarp = 4 * RT, kLoadWarp = 4 * RT + 1;
+    static constexpr int CW = 64 / RT;  // key columns per softmax thread
+    static constexpr int NP = CW / 2;   // float2 pairs per softmax thread
+};
 constexpr uint32_t kTmemCols = 256;
 // tensor-memory column map (per CTA)
 constexpr uint32_t kColO = 0;      // O accumulator, D columns
@@ -96,18 +107,21 @@ __device__ __forceinline__ float div6(float x) {
     return fmaf(r, c, q);
 }
 
-// 32 consecutive fp32 columns of this warp's tensor-memory lanes, as pairs;
-// load and wait in one asm statement (see tmem_ld32).
-__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr, float2 (&v)[16]) {
+// 32 consecutive fp32 columns of this warp's tensor-memory lanes into
+// v[O..O+15] as pairs; load and wait in one asm statement (see tmem_ld32).
+template <int O, int NP>
+__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr, float2 (&v)[NP]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
-        : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x),
-          "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y),
-          "=f"(v[7].x), "=f"(v[7].y), "=f"(v[8].x), "=f"(v[8].y), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[10].x),
-          "=f"(v[10].y), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[13].x),
-          "=f"(v[13].y), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[15].x), "=f"(v[15].y)
+        : "=f"(v[O + 0].x), "=f"(v[O + 0].y), "=f"(v[O + 1].x), "=f"(v[O + 1].y), "=f"(v[O + 2].x),
+          "=f"(v[O + 2].y), "=f"(v[O + 3].x), "=f"(v[O + 3].y), "=f"(v[O + 4].x), "=f"(v[O + 4].y),
+          "=f"(v[O + 5].x), "=f"(v[O + 5].y), "=f"(v[O + 6].x), "=f"(v[O + 6].y), "=f"(v[O + 7].x),
+          "=f"(v[O + 7].y), "=f"(v[O + 8].x), "=f"(v[O + 8].y), "=f"(v[O + 9].x), "=f"(v[O + 9].y),
+          "=f"(v[O + 10].x), "=f"(v[O + 10].y), "=f"(v[O + 11].x), "=f"(v[O + 11].y), "=f"(v[O + 12].x),
+          "=f"(v[O + 12].y), "=f"(v[O + 13].x), "=f"(v[O + 13].y), "=f"(v[O + 14].x), "=f"(v[O + 14].y),
+          "=f"(v[O + 15].x), "=f"(v[O + 15].y)
         : "r"(taddr)
         : "memory");
 }
@@ -138,29 +152,59 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(float2 a, float2 b, float2 c, fl
     return w;
 }
 
-__device__ __forceinline__ float rowmax32f2(const float2 (&v)[16]) {
-    float t[11];
+// Max over the 2*NP values of the pairs v[0..NP) (NP = 16 or 32): a tree of
+// 3-input maxima (all indices are compile-time after unrolling).
+template <int NP>
+__device__ __forceinline__ float pair_val(const float2 (&v)[NP], int k) {
+    return (k & 1) ? v[k >> 1].y : v[k >> 1].x;
+}
+template <int NP>
+__device__ __forceinline__ float rowmax_pairs(const float2 (&v)[NP]) {
+    constexpr int n0 = 2 * NP, n1 = (n0 + 2) / 3;
+    float t[n1];
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-        t[2 * i] = max3f(v[3 * i].x, v[3 * i].y, v[3 * i + 1].x);
-        t[2 * i + 1] = max3f(v[3 * i + 1].y, v[3 * i + 2].x, v[3 * i + 2].y);
+    for (int i = 0; i < n1; ++i) {
+        const int k = 3 * i;
+        const float a = pair_val<NP>(v, k);
+        const float b = k + 1 < n0 ? pair_val<NP>(v, k + 1) : a;
+        const float c = k + 2 < n0 ? pair_val<NP>(v, k + 2) : a;
+        t[i] = max3f(a, b, c);
     }
-    t[10] = fmaxf(v[15].x, v[15].y);
-    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]), u2 = max3f(t[6], t[7], t[8]);
-    return max3f(max3f(u0, u1, u2), t[9], t[10]);
+    int n = n1;
+#pragma unroll
+    for (int round = 0; round < 4; ++round) {
+        if (n > 1) {
+#pragma unroll
+            for (int i = 0; i < (n1 + 2) / 3; ++i) {
+                if (3 * i < n) {
+                    const float a = t[3 * i];
+                    const float b = 3 * i + 1 < n ? t[3 * i + 1] : a;
+                    const float c = 3 * i + 2 < n ? t[3 * i + 2] : a;
+                    t[i] = max3f(a, b, c);
+                }
+            }
+            n = (n + 2) / 3;
+        }
+    }
+    return t[0];
 }
 
 // Max of 16 consecutive values v[b..b+7] (pairs) and 0.
-__device__ __forceinline__ float groupmax16(const float2 (&v)[16], int b) {
+template <int NP>
+__device__ __forceinline__ float groupmax16(const float2 (&v)[NP], int b) {
     const float t0 = max3f(v[b].x, v[b].y, v[b + 1].x), t1 = max3f(v[b + 1].y, v[b + 2].x, v[b + 2].y);
     const float t2 = max3f(v[b + 3].x, v[b + 3].y, v[b + 4].x), t3 = max3f(v[b + 4].y, v[b + 5].x, v[b + 5].y);
     const float t4 = max3f(v[b + 6].x, v[b + 6].y, v[b + 7].x);
     return max3f(max3f(t0, t1, t2), max3f(t3, t4, v[b + 7].y), 0.0f);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
+template <int D, int RT>
+__global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArgs p) {
     using L = Smem<D>;
+    using C = Cfg<RT>;
+    constexpr int kThreads = C::kThreads, kSoftmaxThreads = C::kSoftThreads;
+    constexpr int kMmaWarp = C::kMmaWarp, kLoadWarp = C::kLoadWarp;
+    constexpr int CW = C::CW, NP = C::NP;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
         bar_pv[2], bar_x[4], bar_drain;
@@ -380,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             }
         } else {
             // ================================================== softmax
-            const int quarter = warp & 3, hh = warp >> 2;  // lane quarter, column half
+            const int quarter = warp & 3, hh = warp >> 2;  // lane quarter, column share (0 when RT == 1)
             const int r = 32 * quarter + lane;              // tile row
             const int hf = r >> 6;                          // which query block of the pair
             const int a = hf ? a1 : a0;
@@ -391,11 +435,11 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             float* xmax = reinterpret_cast<float*>(smem + L::xmax);
             const float* rcp_tab = reinterpret_cast<const float*>(smem + L::rcp);
             // Q scale factors of this row into the copy atoms (one per 64 channels)
-            if (hh < D / 64) {
+            for (int ch = hh; ch < D / 64; ch += RT) {
                 uint8_t* atom = smem + L::sfq;
                 const uint8_t* src = p.sfq + ta * (64 * (D / 16)) + (r & 63) * (D / 16);
-                const uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * hh) : 0u;
-                *reinterpret_cast<uint32_t*>(atom + 512 * hh + 16 * (r & 31) + 4 * (r >> 5)) = w;
+                const uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * ch) : 0u;
+                *reinterpret_cast<uint32_t*>(atom + 512 * ch + 16 * (r & 31) + 4 * (r >> 5)) = w;
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar_sfq);
@@ -414,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 mt.ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
                 return mt;
             };
-            float m = -INFINITY, l = 0.0f;  // l: this thread's half of the denominator
+            float m = -INFINITY, l = 0.0f;  // l: this thread's share of the denominator
             bool ok = true;
             StepMeta meta = n_ent > 0 ? load_meta(0) : StepMeta{0, 0.0f, 0.0f};
             for (int j = 0; j < n_ent && ok; ++j) {
@@ -430,9 +474,10 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     break;
                 }
                 tc_fence_after();
-                float2 v[16];
+                float2 v[NP];
                 if (active) {
-                    tmem_ld32x2(lane_base + kColS + 32 * hh, v);
+                    tmem_ld32x2<0>(lane_base + kColS + CW * hh, v);
+                    if (CW == 64) tmem_ld32x2<(NP > 16 ? 16 : 0)>(lane_base + kColS + 32, v);
                 }
                 tc_fence_before();
                 mbar_arrive(&bar_sfree);
@@ -449,35 +494,39 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     const float c2 = ((ph ? gq4 : sq8) * mt.ck) * rdl2e;
                     const float2 c22 = make_float2(c2, c2);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __fmul2_rn(v[i], c22);
-                    const int nk = mt.nk - 32 * hh;  // valid keys among this thread's columns
-                    if (nk < 32) {
-                        if (nk >= 16) {
+                    for (int i = 0; i < NP; ++i) v[i] = __fmul2_rn(v[i], c22);
+                    const int nk = mt.nk - CW * hh;  // valid keys among this thread's columns
+                    if (nk < CW) {
+                        if (nk >= CW - 16) {
 #pragma unroll
-                            for (int i = 8; i < 16; ++i) {
+                            for (int i = NP - 8; i < NP; ++i) {
                                 if (2 * i >= nk) v[i].x = -INFINITY;
                                 if (2 * i + 1 >= nk) v[i].y = -INFINITY;
                             }
                         } else {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
+                            for (int i = 0; i < NP; ++i) {
                                 if (2 * i >= nk) v[i].x = -INFINITY;
                                 if (2 * i + 1 >= nk) v[i].y = -INFINITY;
                             }
                         }
                     }
-                    // row max over both halves: exchange with the partner warp
-                    // (two slots alternating by exchange parity)
-                    float* xm = xmax + (nx & 1) * 256;
-                    xm[hh * 128 + r] = rowmax32f2(v);
-                    mbar_arrive(&bar_x[quarter]);
-                    const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
-                    ++nx;
-                    if (!__all_sync(0xffffffffu, xw)) {
-                        ok = false;
-                        break;
+                    float rmx = rowmax_pairs<NP>(v);
+                    if (RT == 2) {
+                        // row max over both shares: exchange with the partner warp
+                        // (two slots alternating by exchange parity)
+                        float* xm = xmax + (nx & 1) * 256;
+                        xm[hh * 128 + r] = rmx;
+                        mbar_arrive(&bar_x[quarter]);
+                        const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
+                        ++nx;
+                        if (!__all_sync(0xffffffffu, xw)) {
+                            ok = false;
+                            break;
+                        }
+                        rmx = fmaxf(xm[r], xm[128 + r]);
                     }
-                    const float mn = fmaxf(m, fmaxf(xm[r], xm[128 + r]));
+                    const float mn = fmaxf(m, rmx);
                     if (m != -INFINITY && mn > m) {
                         corr = ex2f(m - mn);
                         resc = true;
@@ -487,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     const float2 rt = make_float2(mt.ratio, mt.ratio);
                     float2 acc0 = make_float2(0.0f, 0.0f), acc1 = acc0;
 #pragma unroll
-                    for (int i = 0; i < 16; i += 2) {
+                    for (int i = 0; i < NP; i += 2) {
                         const float2 t0 = __fadd2_rn(v[i], nm), t1 = __fadd2_rn(v[i + 1], nm);
                         const float2 p0 = make_float2(ex2f(t0.x), ex2f(t0.y));
                         const float2 p1 = make_float2(ex2f(t1.x), ex2f(t1.y));
@@ -500,18 +549,18 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                     l = l * corr + (a2.x + a2.y);
                     if (ph == 0) {
 #pragma unroll
-                        for (int ch = 0; ch < 2; ++ch) {
+                        for (int ch = 0; ch < CW / 16; ++ch) {
                             const int b = ch * 8;
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 2 * hh + ch, 64)) =
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 16) * hh + ch, 64)) =
                                 make_uint4(pack_e4m3x4(v[b], v[b + 1]), pack_e4m3x4(v[b + 2], v[b + 3]),
                                            pack_e4m3x4(v[b + 4], v[b + 5]), pack_e4m3x4(v[b + 6], v[b + 7]));
                         }
                     } else {
-                        uint32_t sfw = 0, wq[4];
+                        uint32_t sfw = 0, wq[CW / 8];
 #pragma unroll
-                        for (int gi = 0; gi < 2; ++gi) {
+                        for (int gi = 0; gi < CW / 16; ++gi) {
                             const int b = gi * 8;
-                            const float ym = groupmax16(v, b);
+                            const float ym = groupmax16<NP>(v, b);
                             const uint32_t sf = cvt_e4m3x2(div6(ym), 0.0f) & 0x7Fu;
                             const float rc = rcp_tab[sf];
                             const float2 rc2 = make_float2(rc, rc);
@@ -523,19 +572,29 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                             sfw |= sf << (8 * gi);
                         }
                         // 32 keys = one 16-byte chunk of the 32-byte row
-                        *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, hh, 32)) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
-                        *reinterpret_cast<uint16_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5) + 2 * hh) =
-                            (uint16_t)sfw;
+#pragma unroll
+                        for (int ch = 0; ch < CW / 32; ++ch)
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 32) * hh + ch, 32)) =
+                                make_uint4(wq[4 * ch], wq[4 * ch + 1], wq[4 * ch + 2], wq[4 * ch + 3]);
+                        uint8_t* sfp = pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5);
+                        if (RT == 1) *reinterpret_cast<uint32_t*>(sfp) = sfw;
+                        else *reinterpret_cast<uint16_t*>(sfp + 2 * hh) = (uint16_t)sfw;
                     }
                 } else {
                     // row not in this step: zero weights
                     if (ph == 0) {
 #pragma unroll
-                        for (int ch = 0; ch < 2; ++ch)
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, 2 * hh + ch, 64)) = make_uint4(0, 0, 0, 0);
+                        for (int ch = 0; ch < CW / 16; ++ch)
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 16) * hh + ch, 64)) =
+                                make_uint4(0, 0, 0, 0);
                     } else {
-                        *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, hh, 32)) = make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint16_t*>(pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5) + 2 * hh) = 0;
+#pragma unroll
+                        for (int ch = 0; ch < CW / 32; ++ch)
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 32) * hh + ch, 32)) =
+                                make_uint4(0, 0, 0, 0);
+                        uint8_t* sfp = pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5);
+                        if (RT == 1) *reinterpret_cast<uint32_t*>(sfp) = 0u;
+                        else *reinterpret_cast<uint16_t*>(sfp + 2 * hh) = 0;
                     }
                 }
                 // O rescale (this thread's half of the columns): when the row
@@ -552,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                         tc_fence_after();
                         const uint64_t f2 = need ? pack2(f, f) : pack2(1.0f, 1.0f);
 #pragma unroll 1
-                        for (int c0 = hh * (D / 2); c0 < (hh + 1) * (D / 2); c0 += 32) {
+                        for (int c0 = hh * (D / RT); c0 < (hh + 1) * (D / RT); c0 += 32) {
                             uint32_t o[32];
                             tmem_ld32(lane_base + kColO + c0, o);
 #pragma unroll
@@ -572,8 +631,8 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             }
             // ---- epilogue: both halves of the denominator, then this thread's columns
             ok = __all_sync(0xffffffffu, ok);
-            float lt = 0.0f;
-            {
+            float lt = l;
+            if (RT == 2) {
                 float* xl = xmax + (nx & 1) * 256;
                 xl[hh * 128 + r] = l;
                 mbar_arrive(&bar_x[quarter]);
@@ -600,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 dst += (size_t)(bh / p.H) * p.o0 + (size_t)(bh % p.H) * p.o1 + (size_t)t * p.o2;
             }
 #pragma unroll 1
-            for (int c0 = hh * (D / 2); c0 < (hh + 1) * (D / 2); c0 += 32) {
+            for (int c0 = hh * (D / RT); c0 < (hh + 1) * (D / RT); c0 += 32) {
                 uint32_t o[32];
                 if (have_o) {
                     tmem_ld32(lane_base + kColO + c0, o);
@@ -662,18 +721,20 @@ cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream) {
     const int items = p.B * p.H * ((p.R + 1) / 2);
     if (items == 0) return cudaSuccess;
     const int grid = items < 2 * p.num_sms ? items : 2 * p.num_sms;
+    constexpr int RT = kRowThreads;
+    constexpr int threads = Cfg<RT>::kThreads;
     cudaError_t e = cudaMemsetAsync(p.work_counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
     if (p.d == 64) {
         const size_t smem = attention_smem_bytes<64>(p.R);
-        e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(attention_kernel<64, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attention_kernel<64><<<grid, kThreads, smem, stream>>>(p);
+        attention_kernel<64, RT><<<grid, threads, smem, stream>>>(p);
     } else {
         const size_t smem = attention_smem_bytes<128>(p.R);
-        e = cudaFuncSetAttribute(attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(attention_kernel<128, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attention_kernel<128><<<grid, kThreads, smem, stream>>>(p);
+        attention_kernel<128, RT><<<grid, threads, smem, stream>>>(p);
     }
     return cudaGetLastError();
 }
