@@ -89,14 +89,18 @@ struct Smem {
     static constexpr uint32_t bitmap = p + 2 * p_bytes;        // 4 x 128 words
     static constexpr uint32_t xmax = bitmap + 4 * 128 * 4;     // [2 steps][2 halves][128 rows] floats
     static constexpr uint32_t rcp = xmax + 2 * 2 * 128 * 4;    // 128 floats: 1/value of each ue4m3 code
-    static constexpr uint32_t list = rcp + 128 * 4;            // 2R entries of 16 bits
+    static constexpr uint32_t meta = rcp + 128 * 4;            // kStages StepMeta records (loader -> softmax)
+    static constexpr uint32_t list = meta + kStages * 16;      // 2R entries of 16 bits
 };
 
-// Per-step scalars of a row: key-block size, score scale, value-scale ratio.
-struct StepMeta {
+// Per-step scalars shared by all rows: key-block size, score scale,
+// value-scale ratio.  Written by the loader into the stage's record before it
+// arms the stage barrier; read by the softmax threads after that barrier.
+struct __align__(16) StepMeta {
     int nk;
     float ck;     // K tile scale (FP8) or NVFP4 tile scale
     float ratio;  // V tile scale over the phase unit
+    int pad;
 };
 
 // x / 6 correctly rounded (q = x * RN(1/6), one fma residual correction).
@@ -322,6 +326,8 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             if (lane == 0) {
                 const size_t t0 = (size_t)bh * R + a0;
                 const uint32_t qb8 = 64 * D, qb4 = 32 * D;
+                const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
+                StepMeta* meta_ring = reinterpret_cast<StepMeta*>(smem + L::meta);
                 mbar_expect_tx(&bar_q, (has1 ? 2u : 1u) * (qb8 + qb4));
                 bulk_g2s(smem + L::q8, p.q8 + t0 * qb8, qb8, &bar_q);
                 bulk_g2s(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
@@ -336,6 +342,16 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     const int kb = e & 0xFFF, ph = (e >> 12) & 1;
                     const size_t tk = (size_t)bh * R + kb;
                     uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                    {
+                        StepMeta mt;
+                        mt.nk = p.n_a[kb];
+                        mt.ck = p.scale[(ph ? 4 : 1) * BHR + tk];
+                        const float vs = p.scale[(ph ? 5 : 2) * BHR + tk];
+                        const float sg = ph ? sig4 : sig8;
+                        mt.ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
+                        mt.pad = 0;
+                        meta_ring[st] = mt;  // published by the arrive of the expect_tx below
+                    }
                     if (ph == 0) {
                         mbar_expect_tx(&bar_full[st], 2 * 64 * D);
                         bulk_g2s(sb + L::k_off, p.k8 + tk * (64 * D), 64 * D, &bar_full[st]);
@@ -446,29 +462,22 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             const float sq8 = p.scale[ta], gq4 = p.scale[3 * BHR + ta];
             const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
             const float switch_f = sig4 > 0.0f ? __fdiv_rn(sig8, sig4) : 1.0f;
-            auto load_meta = [&](int j) -> StepMeta {
-                StepMeta mt;
-                const uint32_t e = list[j];
-                const int kb = e & 0xFFF, ph = (e >> 12) & 1;
-                const size_t tk = (size_t)bh * R + kb;
-                mt.nk = p.n_a[kb];
-                mt.ck = p.scale[(ph ? 4 : 1) * BHR + tk];
-                const float vs = p.scale[(ph ? 5 : 2) * BHR + tk];
-                const float sg = ph ? sig4 : sig8;
-                mt.ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
-                return mt;
-            };
+            const StepMeta* meta_ring = reinterpret_cast<const StepMeta*>(smem + L::meta);
+            // row factors of the score scale, in log2 units
+            const float cq8 = sq8 * rdl2e, cq4 = gq4 * rdl2e;
             float m = -INFINITY, l = 0.0f;  // l: this thread's share of the denominator
             bool ok = true;
-            StepMeta meta = n_ent > 0 ? load_meta(0) : StepMeta{0, 0.0f, 0.0f};
             for (int j = 0; j < n_ent && ok; ++j) {
-                const uint32_t g = gstep + j, pb = g & 1;
+                const uint32_t g = gstep + j, pb = g & 1, st = g % kStages;
                 const uint32_t e = list[j];
                 const int ph = (e >> 12) & 1;
                 const bool active = (e >> (13 + hf)) & 1;
+                // S of step g.  Its commit also covers every earlier MMA, in
+                // particular the PV of step g-2, the last reader of P buffer pb.
                 bool waited = mbar_wait(&bar_s, g & 1, abort_v, p.status);
-                // P buffer pb was last read by the PV of step g-2
-                if (waited && g >= 2) waited = mbar_wait(&bar_pv[pb], ((g - 2) >> 1) & 1, abort_v, p.status);
+                // already complete (the S MMA waited for it); acquires the
+                // loader's step record
+                if (waited) waited = mbar_wait(&bar_full[st], (g / kStages) & 1, abort_v, p.status);
                 if (!__all_sync(0xffffffffu, waited)) {
                     ok = false;
                     break;
@@ -481,8 +490,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 }
                 tc_fence_before();
                 mbar_arrive(&bar_sfree);
-                const StepMeta mt = meta;
-                if (j + 1 < n_ent) meta = load_meta(j + 1);  // prefetch the next step's scalars
+                const StepMeta mt = meta_ring[st];
                 uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
                 float corr = 1.0f;
                 bool resc = false;
@@ -491,7 +499,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     // exactly, hence p = 1 exactly, as in the definition: the
                     // product p * ratio then meets the same e4m3 / e2m1
                     // rounding ties as p = e^(s - m) computed exactly.
-                    const float c2 = ((ph ? gq4 : sq8) * mt.ck) * rdl2e;
+                    const float c2 = (ph ? cq4 : cq8) * mt.ck;
                     const float2 c22 = make_float2(c2, c2);
 #pragma unroll
                     for (int i = 0; i < NP; ++i) v[i] = __fmul2_rn(v[i], c22);
