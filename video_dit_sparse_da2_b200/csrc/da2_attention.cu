@@ -65,6 +65,7 @@ constexpr uint32_t kColSfq = 192;  // Q scale factors, 4 columns per 64-channel 
 constexpr uint32_t kColSfk = 200;  // K scale factors, 4 columns
 constexpr uint32_t kColSfp = 204;  // P scale factors, 2 buffers x 4 columns
 constexpr uint32_t kColSfv = 212;  // V scale factors, 2 buffers x 4 columns
+constexpr uint32_t kColMeta = 220; // step record (StepMeta) of the step whose S is in the S buffer
 
 // Step of the merged list: key block (12 bits), phase (1), row mask (2).
 __device__ __forceinline__ uint16_t make_entry(int kb, int phase, int mask) {
@@ -89,13 +90,16 @@ struct Smem {
     static constexpr uint32_t bitmap = p + 2 * p_bytes;        // 4 x 128 words
     static constexpr uint32_t xmax = bitmap + 4 * 128 * 4;     // [2 steps][2 halves][128 rows] floats
     static constexpr uint32_t rcp = xmax + 2 * 2 * 128 * 4;    // 128 floats: 1/value of each ue4m3 code
-    static constexpr uint32_t meta = rcp + 128 * 4;            // kStages StepMeta records (loader -> softmax)
-    static constexpr uint32_t list = meta + kStages * 16;      // 2R entries of 16 bits
+    static constexpr uint32_t meta = rcp + 128 * 4;            // kStages x 32 copies of the StepMeta record
+    static constexpr uint32_t list = meta + kStages * 512;     // 2R entries of 16 bits
 };
 
 // Per-step scalars shared by all rows: key-block size, score scale,
-// value-scale ratio.  Written by the loader into the stage's record before it
-// arms the stage barrier; read by the softmax threads after that barrier.
+// value-scale ratio.  The loader writes 32 copies (one per tensor-memory lane
+// of a quarter) into the stage's 512-byte record before it arms the stage
+// barrier; the MMA thread copies the record into tensor memory next to S
+// (tcgen05.cp, before the S MMA, so the S commit covers it) and the softmax
+// threads load it together with S.
 struct __align__(16) StepMeta {
     int nk;
     float ck;     // K tile scale (FP8) or NVFP4 tile scale
@@ -126,6 +130,45 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t taddr, float2 (&v)[NP]) {
           "=f"(v[O + 10].x), "=f"(v[O + 10].y), "=f"(v[O + 11].x), "=f"(v[O + 11].y), "=f"(v[O + 12].x),
           "=f"(v[O + 12].y), "=f"(v[O + 13].x), "=f"(v[O + 13].y), "=f"(v[O + 14].x), "=f"(v[O + 14].y),
           "=f"(v[O + 15].x), "=f"(v[O + 15].y)
+        : "r"(taddr)
+        : "memory");
+}
+
+// 64 consecutive fp32 columns of this warp's tensor-memory lanes into v[0..31]
+// as pairs, and 4 columns of the step record into r: two loads and one wait
+// in one asm statement.
+__device__ __forceinline__ void tmem_ld64x2_rec(uint32_t taddr, uint32_t raddr, float2 (&v)[32],
+                                                uint32_t (&r)[4]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%68];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%64,%65,%66,%67}, [%69];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x), "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y), "=f"(v[7].x), "=f"(v[7].y), "=f"(v[8].x), "=f"(v[8].y), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[10].x), "=f"(v[10].y), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[13].x), "=f"(v[13].y), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[15].x), "=f"(v[15].y), "=f"(v[16].x), "=f"(v[16].y), "=f"(v[17].x), "=f"(v[17].y), "=f"(v[18].x), "=f"(v[18].y), "=f"(v[19].x), "=f"(v[19].y), "=f"(v[20].x), "=f"(v[20].y), "=f"(v[21].x), "=f"(v[21].y), "=f"(v[22].x), "=f"(v[22].y), "=f"(v[23].x), "=f"(v[23].y), "=f"(v[24].x), "=f"(v[24].y), "=f"(v[25].x), "=f"(v[25].y), "=f"(v[26].x), "=f"(v[26].y), "=f"(v[27].x), "=f"(v[27].y), "=f"(v[28].x), "=f"(v[28].y), "=f"(v[29].x), "=f"(v[29].y), "=f"(v[30].x), "=f"(v[30].y), "=f"(v[31].x), "=f"(v[31].y),
+          "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(taddr), "r"(raddr)
+        : "memory");
+}
+
+// 32 consecutive fp32 columns into v[0..15] as pairs and the 4 columns of the
+// step record into r (two loads, one wait).
+__device__ __forceinline__ void tmem_ld32x2_rec(uint32_t taddr, uint32_t raddr, float2 (&v)[16],
+                                                uint32_t (&r)[4]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%36];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%32,%33,%34,%35}, [%37];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x), "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y), "=f"(v[7].x), "=f"(v[7].y), "=f"(v[8].x), "=f"(v[8].y), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[10].x), "=f"(v[10].y), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[13].x), "=f"(v[13].y), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[15].x), "=f"(v[15].y),
+          "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(taddr), "r"(raddr)
+        : "memory");
+}
+
+// 4 consecutive 32-bit columns of this warp's tensor-memory lanes (load and wait).
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
         : "r"(taddr)
         : "memory");
 }
@@ -216,7 +259,9 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
     __shared__ int abort_sh, item_sh;
     __shared__ int n_ent_sh[2];
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // warp index and everything derived from shared scalars are broadcast
+    // from lane 0 so that the compiler treats them as warp-uniform
+    const int tid = threadIdx.x, warp = warp_uniform(tid >> 5), lane = tid & 31;
     const int R = p.R, BH = p.B * p.H;
     const size_t BHR = (size_t)BH * R;
     const int pairs = (R + 1) / 2;
@@ -255,7 +300,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = tmem_base_sh;
+    const uint32_t tmem = warp_uniform(tmem_base_sh);
 
     uint32_t gstep = 0;         // steps processed by this CTA before the current item
     uint32_t nitem = 0;         // items processed by this CTA
@@ -266,7 +311,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
     for (;;) {
         if (tid == 0) item_sh = atomicAdd(p.work_counter, 1);
         __syncthreads();
-        const int item = item_sh;
+        const int item = warp_uniform(item_sh);
         if (item >= items || *abort_v) break;
         const int bh = item / pairs, pr = item % pairs;
         const int a0 = 2 * pr, a1 = 2 * pr + 1;
@@ -319,125 +364,128 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             }
         }
         __syncthreads();
-        const int n8e = n_ent_sh[0], n_ent = n_ent_sh[0] + n_ent_sh[1];
+        const int n8e = warp_uniform(n_ent_sh[0]), n_ent = warp_uniform(n_ent_sh[0] + n_ent_sh[1]);
 
         if (warp == kLoadWarp) {
-            // ================================================== loader
-            if (lane == 0) {
-                const size_t t0 = (size_t)bh * R + a0;
-                const uint32_t qb8 = 64 * D, qb4 = 32 * D;
-                const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
-                StepMeta* meta_ring = reinterpret_cast<StepMeta*>(smem + L::meta);
-                mbar_expect_tx(&bar_q, (has1 ? 2u : 1u) * (qb8 + qb4));
-                bulk_g2s(smem + L::q8, p.q8 + t0 * qb8, qb8, &bar_q);
-                bulk_g2s(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
-                if (has1) {
-                    bulk_g2s(smem + L::q8 + qb8, p.q8 + (t0 + 1) * qb8, qb8, &bar_q);
-                    bulk_g2s(smem + L::q4 + qb4, p.q4 + (t0 + 1) * qb4, qb4, &bar_q);
+            // ================================================== loader (whole warp, one elected lane issues)
+            const size_t t0 = (size_t)bh * R + a0;
+            const uint32_t qb8 = 64 * D, qb4 = 32 * D;
+            const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
+            mbar_expect_tx_w(&bar_q, (has1 ? 2u : 1u) * (qb8 + qb4));
+            bulk_g2s_w(smem + L::q8, p.q8 + t0 * qb8, qb8, &bar_q);
+            bulk_g2s_w(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
+            if (has1) {
+                bulk_g2s_w(smem + L::q8 + qb8, p.q8 + (t0 + 1) * qb8, qb8, &bar_q);
+                bulk_g2s_w(smem + L::q4 + qb4, p.q4 + (t0 + 1) * qb4, qb4, &bar_q);
+            }
+            for (int j = 0; j < n_ent; ++j) {
+                const uint32_t g = gstep + j, st = g % kStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status)))
+                    break;
+                const uint32_t e = warp_uniform((uint32_t)list[j]);
+                const int kb = e & 0xFFF, ph = (e >> 12) & 1;
+                const size_t tk = (size_t)bh * R + kb;
+                uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                {
+                    // step record: lane i writes copy i (one 16-byte store per lane)
+                    const int nk = p.n_a[kb];
+                    const float ck = p.scale[(ph ? 4 : 1) * BHR + tk];
+                    const float vs = p.scale[(ph ? 5 : 2) * BHR + tk];
+                    const float sg = ph ? sig4 : sig8;
+                    const float ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
+                    reinterpret_cast<uint4*>(smem + L::meta + st * 512)[lane] =
+                        make_uint4((uint32_t)nk, __float_as_uint(ck), __float_as_uint(ratio), 0u);
+                    // visible to the tensor-core copy of the MMA warp, which
+                    // waits on the arrive below
+                    fence_proxy_async_smem();
+                    __syncwarp();
                 }
-                for (int j = 0; j < n_ent; ++j) {
-                    const uint32_t g = gstep + j, st = g % kStages;
-                    if (!mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status)) break;
-                    const uint32_t e = list[j];
-                    const int kb = e & 0xFFF, ph = (e >> 12) & 1;
-                    const size_t tk = (size_t)bh * R + kb;
-                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
-                    {
-                        StepMeta mt;
-                        mt.nk = p.n_a[kb];
-                        mt.ck = p.scale[(ph ? 4 : 1) * BHR + tk];
-                        const float vs = p.scale[(ph ? 5 : 2) * BHR + tk];
-                        const float sg = ph ? sig4 : sig8;
-                        mt.ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
-                        mt.pad = 0;
-                        meta_ring[st] = mt;  // published by the arrive of the expect_tx below
-                    }
-                    if (ph == 0) {
-                        mbar_expect_tx(&bar_full[st], 2 * 64 * D);
-                        bulk_g2s(sb + L::k_off, p.k8 + tk * (64 * D), 64 * D, &bar_full[st]);
-                        bulk_g2s(sb + L::v_off, p.v8 + tk * (64 * D), 64 * D, &bar_full[st]);
-                    } else {
-                        mbar_expect_tx(&bar_full[st], 2 * 32 * D + 1024);
-                        bulk_g2s(sb + L::k_off, p.k4 + tk * (32 * D), 32 * D, &bar_full[st]);
-                        bulk_g2s(sb + L::v_off, p.v4 + tk * (32 * D), 32 * D, &bar_full[st]);
-                        bulk_g2s(sb + L::ksf_off, p.sfk + tk * 512, 512, &bar_full[st]);
-                        bulk_g2s(sb + L::vsf_off, p.sfv + tk * 512, 512, &bar_full[st]);
-                    }
-                    ++loads_issued;
+                if (ph == 0) {
+                    mbar_expect_tx_w(&bar_full[st], 2 * 64 * D);
+                    bulk_g2s_w(sb + L::k_off, p.k8 + tk * (64 * D), 64 * D, &bar_full[st]);
+                    bulk_g2s_w(sb + L::v_off, p.v8 + tk * (64 * D), 64 * D, &bar_full[st]);
+                } else {
+                    mbar_expect_tx_w(&bar_full[st], 2 * 32 * D + 1024);
+                    bulk_g2s_w(sb + L::k_off, p.k4 + tk * (32 * D), 32 * D, &bar_full[st]);
+                    bulk_g2s_w(sb + L::v_off, p.v4 + tk * (32 * D), 32 * D, &bar_full[st]);
+                    bulk_g2s_w(sb + L::ksf_off, p.sfk + tk * 512, 512, &bar_full[st]);
+                    bulk_g2s_w(sb + L::vsf_off, p.sfv + tk * 512, 512, &bar_full[st]);
                 }
+                ++loads_issued;
             }
         } else if (warp == kMmaWarp) {
-            // ================================================== MMA issue
-            if (lane == 0) {
-                bool ok = mbar_wait(&bar_q, nitem & 1, abort_v, p.status);
-                ok = ok && mbar_wait(&bar_sfq, nitem & 1, abort_v, p.status);
-                tc_fence_after();
-                if (ok && n_ent > n8e) {
-                    for (int ch = 0; ch < D / 64; ++ch)
-                        tc_cp_32x128_x4(tmem + kColSfq + 4 * ch, sdesc(smem + L::sfq + 512 * ch, 128, 128));
-                }
-                auto issue_pv = [&](int i) -> bool {
-                    const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
-                    if (!mbar_wait(&bar_p[pb], (g >> 1) & 1, abort_v, p.status)) return false;
-                    tc_fence_after();
-                    const int ph = (list[i] >> 12) & 1;
-                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
-                    uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
-                    if (ph == 0) {
-#pragma unroll
-                        for (int kk = 0; kk < 2; ++kk)
-                            mma_f8(tmem + kColO, sdesc(pbuf + 256 * kk, 128, 512),
-                                   sdesc(sb + L::v_off + 256 * kk, 128, 512), idesc_f8(128, D),
-                                   (i > 0 || kk > 0) ? 1u : 0u);
-                    } else {
-                        tc_cp_32x128_x4(tmem + kColSfp + 4 * pb, sdesc(pbuf + 128 * 64, 128, 128));
-                        tc_cp_32x128_x4(tmem + kColSfv + 4 * pb, sdesc(sb + L::vsf_off, 128, 128));
-                        mma_f4(tmem + kColO, sdesc(pbuf, 128, 256), sdesc(sb + L::v_off, 128, 256), idesc_f4(128, D),
-                               tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
-                    }
-                    tc_commit(&bar_empty[st]);
-                    tc_commit(&bar_pv[pb]);
-                    return true;
-                };
-                for (int j = 0; j < n_ent && ok; ++j) {
-                    const uint32_t g = gstep + j, st = g % kStages;
-                    if (!mbar_wait(&bar_full[st], (g / kStages) & 1, abort_v, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    // the S buffer is free once every softmax thread has read step g-1
-                    if (g > 0 && !mbar_wait(&bar_sfree, (g - 1) & 1, abort_v, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const int ph = (list[j] >> 12) & 1;
-                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
-                    const uint32_t sd = tmem + kColS;
-                    if (ph == 0) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 32; ++kk)
-                            mma_f8(sd, sdesc(smem + L::q8 + 256 * kk, 128, 8 * D),
-                                   sdesc(sb + L::k_off + 256 * kk, 128, 8 * D), idesc_f8(128, 64), kk > 0 ? 1u : 0u);
-                    } else {
-                        tc_cp_32x128_x4(tmem + kColSfk, sdesc(sb + L::ksf_off, 128, 128));
-#pragma unroll
-                        for (int kk = 0; kk < D / 64; ++kk)
-                            mma_f4(sd, sdesc(smem + L::q4 + 256 * kk, 128, 4 * D),
-                                   sdesc(sb + L::k_off + 256 * kk, 128, 4 * D), idesc_f4(128, 64),
-                                   tmem + kColSfq + 4 * kk, tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(&bar_s);
-                    mma_issued = true;
-                    if (j > 0 && !issue_pv(j - 1)) {
-                        ok = false;
-                        break;
-                    }
-                }
-                if (ok && n_ent > 0) ok = issue_pv(n_ent - 1);
-                // S buffer of the last step must be released before the next item's S
-                if (ok && n_ent > 0) mbar_wait(&bar_sfree, (gstep + n_ent - 1) & 1, abort_v, p.status);
+            // ================================================== MMA issue (whole warp, one elected lane issues)
+            auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, p.status));
+            };
+            bool ok = wait_all(&bar_q, nitem & 1);
+            ok = ok && wait_all(&bar_sfq, nitem & 1);
+            tc_fence_after();
+            if (ok && n_ent > n8e) {
+                for (int ch = 0; ch < D / 64; ++ch)
+                    tc_cp_32x128_x4_w(tmem + kColSfq + 4 * ch, sdesc(smem + L::sfq + 512 * ch, 128, 128));
             }
+            auto issue_pv = [&](int i) -> bool {
+                const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
+                if (!wait_all(&bar_p[pb], (g >> 1) & 1)) return false;
+                tc_fence_after();
+                const int ph = (warp_uniform((uint32_t)list[i]) >> 12) & 1;
+                uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
+                if (ph == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        mma_f8_w(tmem + kColO, sdesc(pbuf + 256 * kk, 128, 512), sdesc(sb + L::v_off + 256 * kk, 128, 512),
+                                 idesc_f8(128, D), (i > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                    tc_cp_32x128_x4_w(tmem + kColSfp + 4 * pb, sdesc(pbuf + 128 * 64, 128, 128));
+                    tc_cp_32x128_x4_w(tmem + kColSfv + 4 * pb, sdesc(sb + L::vsf_off, 128, 128));
+                    mma_f4_w(tmem + kColO, sdesc(pbuf, 128, 256), sdesc(sb + L::v_off, 128, 256), idesc_f4(128, D),
+                             tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
+                }
+                tc_commit_w(&bar_empty[st]);
+                tc_commit_w(&bar_pv[pb]);
+                return true;
+            };
+            for (int j = 0; j < n_ent && ok; ++j) {
+                const uint32_t g = gstep + j, st = g % kStages;
+                if (!wait_all(&bar_full[st], (g / kStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                // the S buffer is free once every softmax thread has read step g-1
+                if (g > 0 && !wait_all(&bar_sfree, (g - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int ph = (warp_uniform((uint32_t)list[j]) >> 12) & 1;
+                uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                const uint32_t sd = tmem + kColS;
+                // step record next to S (the previous one was read with S(g-1))
+                tc_cp_32x128_x4_w(tmem + kColMeta, sdesc(smem + L::meta + st * 512, 128, 128));
+                if (ph == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        mma_f8_w(sd, sdesc(smem + L::q8 + 256 * kk, 128, 8 * D), sdesc(sb + L::k_off + 256 * kk, 128, 8 * D),
+                                 idesc_f8(128, 64), kk > 0 ? 1u : 0u);
+                } else {
+                    tc_cp_32x128_x4_w(tmem + kColSfk, sdesc(sb + L::ksf_off, 128, 128));
+#pragma unroll
+                    for (int kk = 0; kk < D / 64; ++kk)
+                        mma_f4_w(sd, sdesc(smem + L::q4 + 256 * kk, 128, 4 * D), sdesc(sb + L::k_off + 256 * kk, 128, 4 * D),
+                                 idesc_f4(128, 64), tmem + kColSfq + 4 * kk, tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit_w(&bar_s);
+                mma_issued = true;
+                if (j > 0 && !issue_pv(j - 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok && n_ent > 0) ok = issue_pv(n_ent - 1);
+            // S buffer of the last step must be released before the next item's S
+            if (ok && n_ent > 0) wait_all(&bar_sfree, (gstep + n_ent - 1) & 1);
         } else {
             // ================================================== softmax
             const int quarter = warp & 3, hh = warp >> 2;  // lane quarter, column share (0 when RT == 1)
@@ -462,35 +510,54 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             const float sq8 = p.scale[ta], gq4 = p.scale[3 * BHR + ta];
             const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
             const float switch_f = sig4 > 0.0f ? __fdiv_rn(sig8, sig4) : 1.0f;
-            const StepMeta* meta_ring = reinterpret_cast<const StepMeta*>(smem + L::meta);
             // row factors of the score scale, in log2 units
             const float cq8 = sq8 * rdl2e, cq4 = gq4 * rdl2e;
             float m = -INFINITY, l = 0.0f;  // l: this thread's share of the denominator
             bool ok = true;
+            uint32_t e_next = n_ent > 0 ? list[0] : 0u;
             for (int j = 0; j < n_ent && ok; ++j) {
-                const uint32_t g = gstep + j, pb = g & 1, st = g % kStages;
-                const uint32_t e = list[j];
+                const uint32_t g = gstep + j, pb = g & 1;
+                const uint32_t e = e_next;
+                if (j + 1 < n_ent) e_next = list[j + 1];
                 const int ph = (e >> 12) & 1;
                 const bool active = (e >> (13 + hf)) & 1;
-                // S of step g.  Its commit also covers every earlier MMA, in
-                // particular the PV of step g-2, the last reader of P buffer pb.
-                bool waited = mbar_wait(&bar_s, g & 1, abort_v, p.status);
-                // already complete (the S MMA waited for it); acquires the
-                // loader's step record
-                if (waited) waited = mbar_wait(&bar_full[st], (g / kStages) & 1, abort_v, p.status);
+                // S of step g and its step record.  The commit also covers every
+                // earlier MMA, in particular the PV of step g-2, the last reader
+                // of P buffer pb.
+                const bool waited = mbar_wait(&bar_s, g & 1, abort_v, p.status);
                 if (!__all_sync(0xffffffffu, waited)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 float2 v[NP];
+                StepMeta mt;
+                float pmax_raw = -INFINITY;  // RT == 2: raw maximum of the partner's columns
                 if (active) {
-                    tmem_ld32x2<0>(lane_base + kColS + CW * hh, v);
-                    if (CW == 64) tmem_ld32x2<(NP > 16 ? 16 : 0)>(lane_base + kColS + 32, v);
+                    uint32_t mw[4];
+                    if constexpr (CW == 64) {
+                        tmem_ld64x2_rec(lane_base + kColS, lane_base + kColMeta, v, mw);
+                    } else {
+                        // the partner warp's columns first, for the row maximum
+                        // only (no exchange between the two warps of a row)
+                        tmem_ld32x2_rec(lane_base + kColS + CW * (1 - hh), lane_base + kColMeta, v, mw);
+                        const int nkp = (int)mw[0] - CW * (1 - hh);
+                        if (nkp < CW) {
+#pragma unroll
+                            for (int i = 0; i < NP; ++i) {
+                                if (2 * i >= nkp) v[i].x = -INFINITY;
+                                if (2 * i + 1 >= nkp) v[i].y = -INFINITY;
+                            }
+                        }
+                        pmax_raw = rowmax_pairs<NP>(v);
+                        tmem_ld32x2<0>(lane_base + kColS + CW * hh, v);
+                    }
+                    mt.nk = (int)mw[0];
+                    mt.ck = __uint_as_float(mw[1]);
+                    mt.ratio = __uint_as_float(mw[2]);
                 }
                 tc_fence_before();
                 mbar_arrive(&bar_sfree);
-                const StepMeta mt = meta_ring[st];
                 uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
                 float corr = 1.0f;
                 bool resc = false;
@@ -521,18 +588,11 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     }
                     float rmx = rowmax_pairs<NP>(v);
                     if (RT == 2) {
-                        // row max over both shares: exchange with the partner warp
-                        // (two slots alternating by exchange parity)
-                        float* xm = xmax + (nx & 1) * 256;
-                        xm[hh * 128 + r] = rmx;
-                        mbar_arrive(&bar_x[quarter]);
-                        const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
-                        ++nx;
-                        if (!__all_sync(0xffffffffu, xw)) {
-                            ok = false;
-                            break;
-                        }
-                        rmx = fmaxf(xm[r], xm[128 + r]);
+                        // The partner scales its columns by the same c2 and
+                        // rounding is monotonic, so the maximum of its scaled
+                        // values is the scaled raw maximum: both warps of the
+                        // row get the same row maximum bit for bit.
+                        if (pmax_raw != -INFINITY) rmx = fmaxf(rmx, pmax_raw * c2);
                     }
                     const float mn = fmaxf(m, rmx);
                     if (m != -INFINITY && mn > m) {
@@ -697,9 +757,9 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
 
     // ---- teardown: drain outstanding async work, then free tensor memory
     __syncthreads();
-    if (warp == kMmaWarp && lane == 0 && mma_issued) {
-        tc_commit(&bar_drain);
-        if (!mbar_wait_drain(&bar_drain, 0)) atomicOr(p.status, DA2_DEV_TIMEOUT);
+    if (warp == kMmaWarp && mma_issued) {
+        tc_commit_w(&bar_drain);
+        if (lane == 0 && !mbar_wait_drain(&bar_drain, 0)) atomicOr(p.status, DA2_DEV_TIMEOUT);
     }
     if (warp == kLoadWarp && lane == 0) {
         // every issued stage fill must have landed before the CTA exits
