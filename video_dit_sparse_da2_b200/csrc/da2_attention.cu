@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             // ================================================== softmax
             const int quarter = warp & 3, hh = warp >> 2;  // lane quarter, column share (0 when RT == 1)
             const int r = 32 * quarter + lane;              // tile row
-            const int hf = r >> 6;                          // which query block of the pair
+            const int hf = quarter >> 1;                    // which query block of the pair (= r >> 6)
             const int a = hf ? a1 : a0;
             const bool qvalid = hf == 0 || has1;
             const size_t ta = (size_t)bh * R + (qvalid ? a : a0);
@@ -514,11 +514,11 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             const float cq8 = sq8 * rdl2e, cq4 = gq4 * rdl2e;
             float m = -INFINITY, l = 0.0f;  // l: this thread's share of the denominator
             bool ok = true;
-            uint32_t e_next = n_ent > 0 ? list[0] : 0u;
+            uint32_t e_next = warp_uniform(n_ent > 0 ? (uint32_t)list[0] : 0u);
             for (int j = 0; j < n_ent && ok; ++j) {
                 const uint32_t g = gstep + j, pb = g & 1;
                 const uint32_t e = e_next;
-                if (j + 1 < n_ent) e_next = list[j + 1];
+                if (j + 1 < n_ent) e_next = warp_uniform((uint32_t)list[j + 1]);
                 const int ph = (e >> 12) & 1;
                 const bool active = (e >> (13 + hf)) & 1;
                 // S of step g and its step record.  The commit also covers every
@@ -603,22 +603,27 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     const float2 nm = make_float2(-mn, -mn);
                     const float2 rt = make_float2(mt.ratio, mt.ratio);
                     float2 acc0 = make_float2(0.0f, 0.0f), acc1 = acc0;
+                    // p = 2^(v - m) and x = p * ratio for the 16 keys b/2.. of a group
+                    auto exp_group = [&](int b) {
 #pragma unroll
-                    for (int i = 0; i < NP; i += 2) {
-                        const float2 t0 = __fadd2_rn(v[i], nm), t1 = __fadd2_rn(v[i + 1], nm);
-                        const float2 p0 = make_float2(ex2f(t0.x), ex2f(t0.y));
-                        const float2 p1 = make_float2(ex2f(t1.x), ex2f(t1.y));
-                        acc0 = __fadd2_rn(acc0, p0);
-                        acc1 = __fadd2_rn(acc1, p1);
-                        v[i] = __fmul2_rn(p0, rt);  // p * ratio
-                        v[i + 1] = __fmul2_rn(p1, rt);
-                    }
-                    const float2 a2 = __fadd2_rn(acc0, acc1);
-                    l = l * corr + (a2.x + a2.y);
+                        for (int i = b; i < b + 8; i += 2) {
+                            const float2 t0 = __fadd2_rn(v[i], nm), t1 = __fadd2_rn(v[i + 1], nm);
+                            const float2 p0 = make_float2(ex2f(t0.x), ex2f(t0.y));
+                            const float2 p1 = make_float2(ex2f(t1.x), ex2f(t1.y));
+                            acc0 = __fadd2_rn(acc0, p0);
+                            acc1 = __fadd2_rn(acc1, p1);
+                            v[i] = __fmul2_rn(p0, rt);
+                            v[i + 1] = __fmul2_rn(p1, rt);
+                        }
+                    };
+                    // Each phase computes and quantizes group by group inside its
+                    // own branch, so the exponentials of one group overlap the
+                    // conversions of the previous one.
                     if (ph == 0) {
 #pragma unroll
                         for (int ch = 0; ch < CW / 16; ++ch) {
                             const int b = ch * 8;
+                            exp_group(b);
                             *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 16) * hh + ch, 64)) =
                                 make_uint4(pack_e4m3x4(v[b], v[b + 1]), pack_e4m3x4(v[b + 2], v[b + 3]),
                                            pack_e4m3x4(v[b + 4], v[b + 5]), pack_e4m3x4(v[b + 6], v[b + 7]));
@@ -628,6 +633,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
 #pragma unroll
                         for (int gi = 0; gi < CW / 16; ++gi) {
                             const int b = gi * 8;
+                            exp_group(b);
                             const float ym = groupmax16<NP>(v, b);
                             const uint32_t sf = cvt_e4m3x2(div6(ym), 0.0f) & 0x7Fu;
                             const float rc = rcp_tab[sf];
@@ -648,6 +654,8 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                         if (RT == 1) *reinterpret_cast<uint32_t*>(sfp) = sfw;
                         else *reinterpret_cast<uint16_t*>(sfp + 2 * hh) = (uint16_t)sfw;
                     }
+                    const float2 a2 = __fadd2_rn(acc0, acc1);
+                    l = l * corr + (a2.x + a2.y);
                 } else {
                     // row not in this step: zero weights
                     if (ph == 0) {
