@@ -45,6 +45,12 @@ namespace da2 {
 namespace {
 
 constexpr int kStages = 3;
+// Of every 8 exponential pairs of a 16-key group, this many are computed on
+// the FMA pipe (exp2_poly) instead of the MUFU unit.
+#ifndef DA2_POLY_PAIRS
+#define DA2_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = DA2_POLY_PAIRS;
 // Softmax threads per row of the tile (1: each thread owns all 64 key columns
 // of a step; 2: two threads split them and exchange the partial row max).
 constexpr int kRowThreads = 1;
@@ -173,6 +179,47 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
         : "memory");
 }
 
+// 64 consecutive 32-bit columns of this warp's lanes (load and wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};"
+                 :
+                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+                 : "memory");
+}
+
+// 2^t (t <= 0, or -inf) for two values on the FMA pipe, an alternative to
+// the MUFU ex2 for part of the weights.  t is clamped to -126 (results stay
+// normal; 2^-126 is far below the smallest weight code), split as n + f with
+// n = round(t) (added to 1.5 * 2^23, whose low mantissa bits then hold n) and
+// f in [-1/2, 1/2]; 2^f = 1 + f * q(f) with q of degree 4 fitted to relative
+// error 2e-7 on that interval (the constant term 1 gives 2^0 = 1 exactly);
+// 2^n is applied by adding n to the exponent field.
+__device__ __forceinline__ float2 exp2_poly(float2 t) {
+    t.x = fmaxf(t.x, -126.0f);
+    t.y = fmaxf(t.y, -126.0f);
+    const float2 big = make_float2(12582912.0f, 12582912.0f);
+    const float2 r = __fadd2_rn(t, big);
+    const float2 n = __fadd2_rn(r, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), t);
+    float2 q = __ffma2_rn(make_float2(1.3264722656e-3f, 1.3264722656e-3f), f,
+                          make_float2(9.6715129912e-3f, 9.6715129912e-3f));
+    q = __ffma2_rn(q, f, make_float2(5.5507335812e-2f, 5.5507335812e-2f));
+    q = __ffma2_rn(q, f, make_float2(2.4022242427e-1f, 2.4022242427e-1f));
+    q = __ffma2_rn(q, f, make_float2(6.9314700365e-1f, 6.9314700365e-1f));
+    float2 p = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+    p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(r.x) << 23));
+    p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(r.y) << 23));
+    return p;
+}
+
 // Four fp32 -> four e4m3 bytes in one word (first value in the low byte).
 __device__ __forceinline__ uint32_t pack_e4m3x4(float2 a, float2 b) {
     uint32_t w;
@@ -236,6 +283,15 @@ __device__ __forceinline__ float rowmax_pairs(const float2 (&v)[NP]) {
     return t[0];
 }
 
+// Max of the 16 consecutive values v[b..b+7] (pairs).
+template <int NP>
+__device__ __forceinline__ float groupmax16_raw(const float2 (&v)[NP], int b) {
+    const float t0 = max3f(v[b].x, v[b].y, v[b + 1].x), t1 = max3f(v[b + 1].y, v[b + 2].x, v[b + 2].y);
+    const float t2 = max3f(v[b + 3].x, v[b + 3].y, v[b + 4].x), t3 = max3f(v[b + 4].y, v[b + 5].x, v[b + 5].y);
+    const float t4 = max3f(v[b + 6].x, v[b + 6].y, v[b + 7].x);
+    return max3f(max3f(t0, t1, t2), t3, fmaxf(t4, v[b + 7].y));
+}
+
 // Max of 16 consecutive values v[b..b+7] (pairs) and 0.
 template <int NP>
 __device__ __forceinline__ float groupmax16(const float2 (&v)[NP], int b) {
@@ -253,8 +309,11 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
     constexpr int kMmaWarp = C::kMmaWarp, kLoadWarp = C::kLoadWarp;
     constexpr int CW = C::CW, NP = C::NP;
     extern __shared__ __align__(1024) uint8_t smem[];
+    // bar_empty[st] completes when the PV of a step in stage st has finished:
+    // it frees the stage for the loader and tells the softmax threads that O
+    // holds that step
     __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
-        bar_pv[2], bar_x[4], bar_drain;
+        bar_x[4], bar_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh, item_sh;
     __shared__ int n_ent_sh[2];
@@ -282,7 +341,6 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
         mbar_init(&bar_sfree, kSoftmaxThreads);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar_p[s], kSoftmaxThreads);
-            mbar_init(&bar_pv[s], 1);
         }
         for (int s = 0; s < 4; ++s) mbar_init(&bar_x[s], 64);  // the two warps of a row quarter
         mbar_init(&bar_drain, 1);
@@ -425,26 +483,39 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 for (int ch = 0; ch < D / 64; ++ch)
                     tc_cp_32x128_x4_w(tmem + kColSfq + 4 * ch, sdesc(smem + L::sfq + 512 * ch, 128, 128));
             }
+            // Descriptors of the fixed buffers; a stage or P buffer is selected
+            // by adding its byte offset / 16 to the start-address field (bits
+            // 0-13, which hold the shared-memory address / 16 without carry
+            // since shared memory ends below 256 KB).
+            const uint64_t dq8 = sdesc(smem + L::q8, 128, 8 * D), dq4 = sdesc(smem + L::q4, 128, 4 * D);
+            const uint64_t dk8 = sdesc(smem + L::stage + L::k_off, 128, 8 * D);
+            const uint64_t dk4 = sdesc(smem + L::stage + L::k_off, 128, 4 * D);
+            const uint64_t dv8 = sdesc(smem + L::stage + L::v_off, 128, 512);
+            const uint64_t dv4 = sdesc(smem + L::stage + L::v_off, 128, 256);
+            const uint64_t dksf = sdesc(smem + L::stage + L::ksf_off, 128, 128);
+            const uint64_t dvsf = sdesc(smem + L::stage + L::vsf_off, 128, 128);
+            const uint64_t dmeta = sdesc(smem + L::meta, 128, 128);
+            const uint64_t dp8 = sdesc(smem + L::p, 128, 512), dp4 = sdesc(smem + L::p, 128, 256);
+            const uint64_t dpsf = sdesc(smem + L::p + 128 * 64, 128, 128);
             auto issue_pv = [&](int i) -> bool {
                 const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
                 if (!wait_all(&bar_p[pb], (g >> 1) & 1)) return false;
                 tc_fence_after();
                 const int ph = (warp_uniform((uint32_t)list[i]) >> 12) & 1;
-                uint8_t* sb = smem + L::stage + st * L::stage_bytes;
-                uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
+                const uint64_t so = (st * L::stage_bytes) >> 4, po = (pb * L::p_bytes) >> 4;
                 if (ph == 0) {
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
-                        mma_f8_w(tmem + kColO, sdesc(pbuf + 256 * kk, 128, 512), sdesc(sb + L::v_off + 256 * kk, 128, 512),
-                                 idesc_f8(128, D), (i > 0 || kk > 0) ? 1u : 0u);
+                        mma_f8_w(tmem + kColO, dp8 + po + 16 * kk, dv8 + so + 16 * kk, idesc_f8(128, D),
+                                 (i > 0 || kk > 0) ? 1u : 0u);
                 } else {
-                    tc_cp_32x128_x4_w(tmem + kColSfp + 4 * pb, sdesc(pbuf + 128 * 64, 128, 128));
-                    tc_cp_32x128_x4_w(tmem + kColSfv + 4 * pb, sdesc(sb + L::vsf_off, 128, 128));
-                    mma_f4_w(tmem + kColO, sdesc(pbuf, 128, 256), sdesc(sb + L::v_off, 128, 256), idesc_f4(128, D),
-                             tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
+                    tc_cp_32x128_x4_w(tmem + kColSfp + 4 * pb, dpsf + po);
+                    tc_cp_32x128_x4_w(tmem + kColSfv + 4 * pb, dvsf + so);
+                    mma_f4_w(tmem + kColO, dp4 + po, dv4 + so, idesc_f4(128, D), tmem + kColSfp + 4 * pb,
+                             tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
                 }
+                // frees the stage and tells the softmax threads that O holds step g
                 tc_commit_w(&bar_empty[st]);
-                tc_commit_w(&bar_pv[pb]);
                 return true;
             };
             for (int j = 0; j < n_ent && ok; ++j) {
@@ -460,21 +531,20 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 }
                 tc_fence_after();
                 const int ph = (warp_uniform((uint32_t)list[j]) >> 12) & 1;
-                uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                const uint64_t so = (st * L::stage_bytes) >> 4;
                 const uint32_t sd = tmem + kColS;
                 // step record next to S (the previous one was read with S(g-1))
-                tc_cp_32x128_x4_w(tmem + kColMeta, sdesc(smem + L::meta + st * 512, 128, 128));
+                tc_cp_32x128_x4_w(tmem + kColMeta, dmeta + st * (512 >> 4));
                 if (ph == 0) {
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
-                        mma_f8_w(sd, sdesc(smem + L::q8 + 256 * kk, 128, 8 * D), sdesc(sb + L::k_off + 256 * kk, 128, 8 * D),
-                                 idesc_f8(128, 64), kk > 0 ? 1u : 0u);
+                        mma_f8_w(sd, dq8 + 16 * kk, dk8 + so + 16 * kk, idesc_f8(128, 64), kk > 0 ? 1u : 0u);
                 } else {
-                    tc_cp_32x128_x4_w(tmem + kColSfk, sdesc(sb + L::ksf_off, 128, 128));
+                    tc_cp_32x128_x4_w(tmem + kColSfk, dksf + so);
 #pragma unroll
                     for (int kk = 0; kk < D / 64; ++kk)
-                        mma_f4_w(sd, sdesc(smem + L::q4 + 256 * kk, 128, 4 * D), sdesc(sb + L::k_off + 256 * kk, 128, 4 * D),
-                                 idesc_f4(128, 64), tmem + kColSfq + 4 * kk, tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
+                        mma_f4_w(sd, dq4 + 16 * kk, dk4 + so + 16 * kk, idesc_f4(128, 64), tmem + kColSfq + 4 * kk,
+                                 tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
                 }
                 tc_commit_w(&bar_s);
                 mma_issued = true;
@@ -586,7 +656,16 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                             }
                         }
                     }
-                    float rmx = rowmax_pairs<NP>(v);
+                    // maxima of the 16-key groups (they also give the NVFP4
+                    // group scales below) and of the row
+                    constexpr int NGR = CW / 16;
+                    float gm[NGR];
+#pragma unroll
+                    for (int gi = 0; gi < NGR; ++gi) gm[gi] = groupmax16_raw<NP>(v, 8 * gi);
+                    float rmx = gm[0];
+#pragma unroll
+                    for (int gi = 1; gi < NGR; gi += 2)
+                        rmx = gi + 1 < NGR ? max3f(rmx, gm[gi], gm[gi + 1]) : fmaxf(rmx, gm[gi]);
                     if (RT == 2) {
                         // The partner scales its columns by the same c2 and
                         // rounding is monotonic, so the maximum of its scaled
@@ -603,13 +682,13 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     const float2 nm = make_float2(-mn, -mn);
                     const float2 rt = make_float2(mt.ratio, mt.ratio);
                     float2 acc0 = make_float2(0.0f, 0.0f), acc1 = acc0;
-                    // p = 2^(v - m) and x = p * ratio for the 16 keys b/2.. of a group
+                    // p = 2^(v - m) and x = p * ratio for the 16 keys of a group (b = first pair)
                     auto exp_group = [&](int b) {
 #pragma unroll
                         for (int i = b; i < b + 8; i += 2) {
                             const float2 t0 = __fadd2_rn(v[i], nm), t1 = __fadd2_rn(v[i + 1], nm);
-                            const float2 p0 = make_float2(ex2f(t0.x), ex2f(t0.y));
-                            const float2 p1 = make_float2(ex2f(t1.x), ex2f(t1.y));
+                            const float2 p0 = ((i - b) < kPolyPairs) ? exp2_poly(t0) : make_float2(ex2f(t0.x), ex2f(t0.y));
+                            const float2 p1 = ((i + 1 - b) < kPolyPairs) ? exp2_poly(t1) : make_float2(ex2f(t1.x), ex2f(t1.y));
                             acc0 = __fadd2_rn(acc0, p0);
                             acc1 = __fadd2_rn(acc1, p1);
                             v[i] = __fmul2_rn(p0, rt);
@@ -629,21 +708,30 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                                            pack_e4m3x4(v[b + 4], v[b + 5]), pack_e4m3x4(v[b + 6], v[b + 7]));
                         }
                     } else {
+                        // Group scale from the group maximum: p is monotonic in v
+                        // and rounding is monotonic, so the largest weight of the
+                        // group is 2^(max v - m) * ratio rounded as each weight
+                        // is.  Scale code and 1/value are known before the
+                        // weights; each weight is then (p * ratio) * 1/value.
                         uint32_t sfw = 0, wq[CW / 8];
+                        float rcs[NGR];
 #pragma unroll
-                        for (int gi = 0; gi < CW / 16; ++gi) {
+                        for (int gi = 0; gi < NGR; ++gi) {
+                            const float ym = ex2f(gm[gi] - m) * mt.ratio;
+                            const uint32_t sf = cvt_e4m3x2(div6(ym), 0.0f);
+                            rcs[gi] = rcp_tab[sf];  // 0 for code 0: every weight of the group 0
+                            sfw |= sf << (8 * gi);
+                        }
+#pragma unroll
+                        for (int gi = 0; gi < NGR; ++gi) {
                             const int b = gi * 8;
                             exp_group(b);
-                            const float ym = groupmax16<NP>(v, b);
-                            const uint32_t sf = cvt_e4m3x2(div6(ym), 0.0f) & 0x7Fu;
-                            const float rc = rcp_tab[sf];
-                            const float2 rc2 = make_float2(rc, rc);
+                            const float2 rc2 = make_float2(rcs[gi], rcs[gi]);
                             float2 y[8];
 #pragma unroll
                             for (int i = 0; i < 8; ++i) y[i] = __fmul2_rn(v[b + i], rc2);
-                            wq[2 * gi] = sf ? pack_e2m1x8(y[0], y[1], y[2], y[3]) : 0u;
-                            wq[2 * gi + 1] = sf ? pack_e2m1x8(y[4], y[5], y[6], y[7]) : 0u;
-                            sfw |= sf << (8 * gi);
+                            wq[2 * gi] = pack_e2m1x8(y[0], y[1], y[2], y[3]);
+                            wq[2 * gi + 1] = pack_e2m1x8(y[4], y[5], y[6], y[7]);
                         }
                         // 32 keys = one 16-byte chunk of the 32-byte row
 #pragma unroll
@@ -681,22 +769,35 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 const bool need = (resc || sw) && j > 0;
                 if (__any_sync(0xffffffffu, need)) {
                     // O must hold the PV of step g-1 first
-                    const bool w2 = mbar_wait(&bar_pv[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_v, p.status);
+                    const bool w2 = mbar_wait(&bar_empty[(g - 1) % kStages], ((g - 1) / kStages) & 1, abort_v, p.status);
                     if (!__all_sync(0xffffffffu, w2)) ok = false;
                     if (ok) {
                         tc_fence_after();
                         const uint64_t f2 = need ? pack2(f, f) : pack2(1.0f, 1.0f);
+                        // this thread's D/RT columns of O, in 64-column round trips
+                        // (32 when it owns only 32)
+                        constexpr int OW = (RT == 1 && (D / RT) % 64 == 0) ? 64 : 32;
 #pragma unroll 1
-                        for (int c0 = hh * (D / RT); c0 < (hh + 1) * (D / RT); c0 += 32) {
-                            uint32_t o[32];
-                            tmem_ld32(lane_base + kColO + c0, o);
+                        for (int c0 = hh * (D / RT); c0 < (hh + 1) * (D / RT); c0 += OW) {
+                            uint32_t o[64];
+                            if constexpr (OW == 64) {
+                                tmem_ld64(lane_base + kColO + c0, o);
+                            } else {
+                                uint32_t (&o32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+                                tmem_ld32(lane_base + kColO + c0, o32);
+                            }
 #pragma unroll
-                            for (int c = 0; c < 32; c += 2) {
+                            for (int c = 0; c < OW; c += 2) {
                                 const uint64_t v = mul2(pack2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), f2);
                                 o[c] = __float_as_uint(lo2(v));
                                 o[c + 1] = __float_as_uint(hi2(v));
                             }
-                            tmem_st32(lane_base + kColO + c0, o);
+                            if constexpr (OW == 64) {
+                                tmem_st64(lane_base + kColO + c0, o);
+                            } else {
+                                const uint32_t (&o32)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&o[0]);
+                                tmem_st32(lane_base + kColO + c0, o32);
+                            }
                         }
                         tc_wait_st();
                     }
@@ -721,7 +822,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             const bool have = n_ent > 0 && ok;
             if (have) {
                 const uint32_t g = gstep + n_ent - 1;
-                if (!mbar_wait(&bar_pv[g & 1], (g >> 1) & 1, abort_v, p.status)) ok = false;
+                if (!mbar_wait(&bar_empty[g % kStages], (g / kStages) & 1, abort_v, p.status)) ok = false;
                 tc_fence_after();
                 const float unit = n_ent > n8e ? sig4 : sig8;
                 o_scale = lt > 0.0f ? __fdiv_rn(unit, lt) : 0.0f;
