@@ -241,7 +241,7 @@ def oracle_sample(w, budget_s: float = 20.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=250)  # about 1 s timed on the default workload
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="wan2.1-1.3b-480p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
