@@ -27,6 +27,29 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ms/call and dense-equiv TFLOPS at 1 B200; % of mixed FP8/FP4 tensor roofline"
+
+# DRAM bytes (read + write) of one attention launch, from the ncu capture in
+# profiles/attention_kernel_wan13b_480p.md, valid for the attention sources
+# whose hash is given (the field is null for any other source or workload).
+ATTN_TRAFFIC = {"wan2.1-1.3b-480p": {"sources_sha256_16": "01729b12788121a3", "bytes": 146748928 + 67008256}}
+_ATTN_SOURCES = ("video_dit_sparse_da2_b200/csrc/da2_attention.cu", "video_dit_sparse_da2_b200/csrc/da2_common.cuh")
+
+
+def attention_traffic(workload: str):
+    import hashlib
+    rec = ATTN_TRAFFIC.get(workload)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    root = os.path.dirname(os.path.abspath(__file__))
+    try:
+        for f in _ATTN_SOURCES:
+            with open(os.path.join(root, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return rec["bytes"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
+
 UNIT = "TFLOPS (dense-equivalent, whole job)"
 
 
@@ -311,7 +334,8 @@ def main():
         "config": config,
         "ms_per_call": {"prepare": r["t_prep"], "plan": r["t_plan"], "attention": r["t_attn"], "total": ms},
         "roofline": {"bound": "tensor", "kernel": "attention", "achieved": achieved, "peak": peak_mix,
-                     "unit": "TFLOP/s", "frac": achieved / peak_mix if peak_mix else None, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak_mix if peak_mix else None,
+                     "traffic": attention_traffic(w.name),
                      "peak_source": f"{peaks['source']} bf16 {peaks['bf16_tflops']} TF x2 (FP8) / x4 (NVFP4), "
                                     f"mixed by the kept FP8/NVFP4 FLOPs",
                      "fp8_tflop": F8 / 1e12, "fp4_tflop": F4 / 1e12},
