@@ -48,66 +48,106 @@ __device__ __forceinline__ double exp_fixed(double x) {
 }
 
 // ---------------------------------------------------------------- logits
-// 64 x 64 output tile of both branches per CTA; each thread owns 4 x 4
-// outputs per branch and accumulates them in ascending channel order.
-template <int D>
-__global__ void __launch_bounds__(256) logits_kernel(PlanArgs p, double rd) {
-    __shared__ double sQa[16][64], sQm[16][64], sKa[16][64], sKm[16][64];
-    const int R = p.R, bh = blockIdx.z;
-    const int a0 = blockIdx.y * 64, b0 = blockIdx.x * 64;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const size_t plane = (size_t)p.BH * R * D;
-    const double* Qa = p.desc + 0 * plane + (size_t)bh * R * D;
-    const double* Qm = p.desc + 1 * plane + (size_t)bh * R * D;
-    const double* Ka = p.desc + 2 * plane + (size_t)bh * R * D;
-    const double* Km = p.desc + 3 * plane + (size_t)bh * R * D;
-    double acc_a[4][4], acc_m[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc_a[i][j] = acc_m[i][j] = 0.0;
+// One branch (average or max descriptors) of one head per CTA, 128 x 128
+// output tile; each thread owns 8 x 8 outputs: rows {2ty, 2ty+1} + 32 i and
+// columns {2tx, 2tx+1} + 32 j (i, j < 4), so that the 16-byte shared-memory
+// reads of a warp are contiguous.  Channels are staged 16 at a time
+// (transposed, [channel][row]) in two shared buffers; every output is one fma
+// chain over c = 0..d-1 in ascending order starting from 0, as defined.
+constexpr int kLgTile = 128, kLgKc = 16, kLgThreads = 256;
+constexpr size_t kLgSmem = 2ull * 2 * kLgKc * kLgTile * sizeof(double);  // 64 KB
 
-    for (int k0 = 0; k0 < D; k0 += 16) {
-        for (int i = threadIdx.x; i < 64 * 16; i += 256) {
-            const int r = i >> 4, c = i & 15;
-            const int ra = a0 + r, rb = b0 + r;
-            sQa[c][r] = ra < R ? Qa[(size_t)ra * D + k0 + c] : 0.0;
-            sQm[c][r] = ra < R ? Qm[(size_t)ra * D + k0 + c] : 0.0;
-            sKa[c][r] = rb < R ? Ka[(size_t)rb * D + k0 + c] : 0.0;
-            sKm[c][r] = rb < R ? Km[(size_t)rb * D + k0 + c] : 0.0;
-        }
-        __syncthreads();
+template <int D>
+__global__ void __launch_bounds__(kLgThreads, 1) logits_kernel(PlanArgs p, double rd) {
+    extern __shared__ __align__(16) double lg_smem[];
+    double* sQ = lg_smem;                          // [2][kLgKc][kLgTile]
+    double* sK = lg_smem + 2 * kLgKc * kLgTile;    // [2][kLgKc][kLgTile]
+    const int R = p.R, bh = blockIdx.z >> 1, branch = blockIdx.z & 1;
+    const int a0 = blockIdx.y * kLgTile, b0 = blockIdx.x * kLgTile;
+    const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+    const size_t plane = (size_t)p.BH * R * D;
+    const double* Qs = p.desc + (size_t)branch * plane + (size_t)bh * R * D;
+    const double* Ks = p.desc + (size_t)(2 + branch) * plane + (size_t)bh * R * D;
+
+    // staging: thread t moves channel pairs of rows (t + 256 it) % 128
+    double2 rq[4], rk[4];
+    auto fetch = [&](int k0) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            double qa[4], qm[4], ka[4], km[4];
+        for (int it = 0; it < 4; ++it) {
+            const int idx = it * kLgThreads + t, row = idx & (kLgTile - 1), cp = idx >> 7;
+            const int ra = a0 + row, rb = b0 + row;
+            rq[it] = ra < R ? *reinterpret_cast<const double2*>(Qs + (size_t)ra * D + k0 + 2 * cp)
+                            : make_double2(0.0, 0.0);
+            rk[it] = rb < R ? *reinterpret_cast<const double2*>(Ks + (size_t)rb * D + k0 + 2 * cp)
+                            : make_double2(0.0, 0.0);
+        }
+    };
+    auto stage = [&](int buf) {
+        double* q = sQ + buf * kLgKc * kLgTile;
+        double* k = sK + buf * kLgKc * kLgTile;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = it * kLgThreads + t, row = idx & (kLgTile - 1), cp = idx >> 7;
+            q[(2 * cp) * kLgTile + row] = rq[it].x;
+            q[(2 * cp + 1) * kLgTile + row] = rq[it].y;
+            k[(2 * cp) * kLgTile + row] = rk[it].x;
+            k[(2 * cp + 1) * kLgTile + row] = rk[it].y;
+        }
+    };
+
+    double acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+
+    fetch(0);
+    stage(0);
+    __syncthreads();
+    constexpr int NCH = D / kLgKc;
+#pragma unroll 1
+    for (int ch = 0; ch < NCH; ++ch) {
+        const int buf = ch & 1;
+        if (ch + 1 < NCH) fetch((ch + 1) * kLgKc);  // global loads in flight during the FMAs
+        const double* q = sQ + buf * kLgKc * kLgTile;
+        const double* k = sK + buf * kLgKc * kLgTile;
+#pragma unroll
+        for (int c = 0; c < kLgKc; ++c) {
+            double qa[8], kb[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                qa[i] = sQa[c][ty * 4 + i];
-                qm[i] = sQm[c][ty * 4 + i];
-                ka[i] = sKa[c][tx * 4 + i];
-                km[i] = sKm[c][tx * 4 + i];
+                const double2 x = *reinterpret_cast<const double2*>(q + c * kLgTile + 32 * i + 2 * ty);
+                const double2 y = *reinterpret_cast<const double2*>(k + c * kLgTile + 32 * i + 2 * tx);
+                qa[2 * i] = x.x;
+                qa[2 * i + 1] = x.y;
+                kb[2 * i] = y.x;
+                kb[2 * i + 1] = y.y;
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc_a[i][j] = fma(qa[i], ka[j], acc_a[i][j]);
-                    acc_m[i][j] = fma(qm[i], km[j], acc_m[i][j]);
-                }
+                for (int j = 0; j < 8; ++j) acc[i][j] = fma(qa[i], kb[j], acc[i][j]);
         }
-        __syncthreads();
+        if (ch + 1 < NCH) {
+            stage(buf ^ 1);  // the other buffer was last read before the previous barrier
+            __syncthreads();
+        }
     }
+    double* out = branch ? p.Lmax : p.A;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int a = a0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int a = a0 + 32 * (i >> 1) + 2 * ty + (i & 1);
         if (a >= R) continue;
+        double* orow = out + ((size_t)bh * R + a) * R;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int b = b0 + tx * 4 + j;
-            if (b >= R) continue;
-            const size_t o = ((size_t)bh * R + a) * R + b;
-            p.A[o] = acc_a[i][j] * rd;
-            p.Lmax[o] = acc_m[i][j] * rd;
+        for (int j = 0; j < 8; j += 2) {
+            const int b = b0 + 32 * (j >> 1) + 2 * tx;
+            if (b + 1 < R && ((R & 1) == 0)) {
+                *reinterpret_cast<double2*>(orow + b) = make_double2(acc[i][j] * rd, acc[i][j + 1] * rd);
+            } else {
+                if (b < R) orow[b] = acc[i][j] * rd;
+                if (b + 1 < R) orow[b + 1] = acc[i][j + 1] * rd;
+            }
         }
     }
 }
@@ -415,9 +455,18 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     const long long T8 = RR * p.bp8 / 10000, Tk = RR * (p.bp8 + p.bp4) / 10000;
     cudaError_t e;
     const double rd = 1.0 / sqrt((double)p.d);
-    dim3 lg((R + 63) / 64, (R + 63) / 64, BH);
-    if (p.d == 64) logits_kernel<64><<<lg, 256, 0, stream>>>(p, rd);
-    else logits_kernel<128><<<lg, 256, 0, stream>>>(p, rd);
+    dim3 lg((R + kLgTile - 1) / kLgTile, (R + kLgTile - 1) / kLgTile, 2 * BH);
+    if (p.d == 64) {
+        if ((e = cudaFuncSetAttribute(logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLgSmem)) !=
+            cudaSuccess)
+            return e;
+        logits_kernel<64><<<lg, kLgThreads, kLgSmem, stream>>>(p, rd);
+    } else {
+        if ((e = cudaFuncSetAttribute(logits_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLgSmem)) !=
+            cudaSuccess)
+            return e;
+        logits_kernel<128><<<lg, kLgThreads, kLgSmem, stream>>>(p, rd);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.abits_minmax, 0xFF, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.abits_minmax + BH, 0, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
