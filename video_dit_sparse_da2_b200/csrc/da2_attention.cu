@@ -338,9 +338,9 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             mbar_init(&bar_empty[s], 1);
         }
         mbar_init(&bar_s, 1);
-        mbar_init(&bar_sfree, kSoftmaxThreads);
+        mbar_init(&bar_sfree, kSoftmaxThreads / 32);  // one arrive per softmax warp
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar_p[s], kSoftmaxThreads);
+            mbar_init(&bar_p[s], kSoftmaxThreads / 32);
         }
         for (int s = 0; s < 4; ++s) mbar_init(&bar_x[s], 64);  // the two warps of a row quarter
         mbar_init(&bar_drain, 1);
@@ -626,8 +626,11 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     mt.ck = __uint_as_float(mw[1]);
                     mt.ratio = __uint_as_float(mw[2]);
                 }
+                // the warp's loads of S are complete (their wait is warp-wide):
+                // one arrive per warp
                 tc_fence_before();
-                mbar_arrive(&bar_sfree);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sfree);
                 uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
                 float corr = 1.0f;
                 bool resc = false;
@@ -711,8 +714,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                         // Group scale from the group maximum: p is monotonic in v
                         // and rounding is monotonic, so the largest weight of the
                         // group is 2^(max v - m) * ratio rounded as each weight
-                        // is.  Scale code and 1/value are known before the
-                        // weights; each weight is then (p * ratio) * 1/value.
+                        // is.  Scale code and 1/value are known before the weights.
                         uint32_t sfw = 0, wq[CW / 8];
                         float rcs[NGR];
 #pragma unroll
@@ -722,14 +724,22 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                             rcs[gi] = rcp_tab[sf];  // 0 for code 0: every weight of the group 0
                             sfw |= sf << (8 * gi);
                         }
+                        // weights p * (ratio * 1/value): the same value as
+                        // (p * ratio) * 1/value when p is a power of two, in
+                        // particular p = 1 for the row maximum
 #pragma unroll
                         for (int gi = 0; gi < NGR; ++gi) {
-                            const int b = gi * 8;
-                            exp_group(b);
-                            const float2 rc2 = make_float2(rcs[gi], rcs[gi]);
+                            const float sgv = mt.ratio * rcs[gi];
+                            const float2 sg2 = make_float2(sgv, sgv);
                             float2 y[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) y[i] = __fmul2_rn(v[b + i], rc2);
+                            for (int i = 0; i < 8; ++i) {
+                                const float2 tt = __fadd2_rn(v[8 * gi + i], nm);
+                                const float2 pp = i < kPolyPairs ? exp2_poly(tt) : make_float2(ex2f(tt.x), ex2f(tt.y));
+                                if (i & 1) acc1 = __fadd2_rn(acc1, pp);
+                                else acc0 = __fadd2_rn(acc0, pp);
+                                y[i] = __fmul2_rn(pp, sg2);
+                            }
                             wq[2 * gi] = pack_e2m1x8(y[0], y[1], y[2], y[3]);
                             wq[2 * gi + 1] = pack_e2m1x8(y[4], y[5], y[6], y[7]);
                         }
@@ -802,9 +812,12 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                         tc_wait_st();
                     }
                 }
+                // every thread makes its weight stores visible to the tensor
+                // core; after the warp barrier one lane publishes them
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&bar_p[pb]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_p[pb]);
             }
             // ---- epilogue: both halves of the denominator, then this thread's columns
             ok = __all_sync(0xffffffffu, ok);
