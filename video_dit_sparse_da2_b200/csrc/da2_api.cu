@@ -219,6 +219,7 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
     a.cnt = plan->cnt;
     a.kidx = plan->kidx;
     a.status = h->d_status;
+    a.num_sms = h->num_sms;
     da2::plan_carve_scratch(&a, plan->scratch);
     cudaError_t e = da2::launch_plan(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DA2_OK : cuda_fail(e);

@@ -157,7 +157,7 @@ __device__ __forceinline__ void tmem_ld64x2_rec(uint32_t taddr, uint32_t raddr, 
 
 // 32 consecutive fp32 columns into v[0..15] as pairs and the 4 columns of the
 // step record into r (two loads, one wait).
-__device__ __forceinline__ void tmem_ld32x2_rec(uint32_t taddr, uint32_t raddr, float2 (&v)[16],
+[[maybe_unused]] __device__ __forceinline__ void tmem_ld32x2_rec(uint32_t taddr, uint32_t raddr, float2 (&v)[16],
                                                 uint32_t (&r)[4]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%36];\n\t"
@@ -170,7 +170,7 @@ __device__ __forceinline__ void tmem_ld32x2_rec(uint32_t taddr, uint32_t raddr, 
 }
 
 // 4 consecutive 32-bit columns of this warp's tensor-memory lanes (load and wait).
-__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+[[maybe_unused]] __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n\t"
         "tcgen05.wait::ld.sync.aligned;"

@@ -21,14 +21,16 @@ cudaError_t launch_prepare(const PrepareArgs& p, cudaStream_t stream);
 
 // Per head and per quota target, the state of the radix selection of the
 // T-th largest 96-bit key (A bits : ~pair index).
-struct SelectTarget {
+struct __align__(16) SelectTarget {
     unsigned long long p_hi;  // selected prefix, left aligned in 96 bits
     unsigned int p_lo;
     int nbits;                // bits of the key already fixed
     long long need;           // rank still sought inside the current prefix (1-based)
     int unique;               // the current prefix holds exactly one key: record it next pass
+    int found;                // that key was recorded (the pass's scan then marks the target done)
     int done;                 // threshold known (or no threshold: none)
     int none;                 // T == 0: nothing gets this precision or better
+    long long matches;        // keys that match the current prefix
     unsigned long long key_hi;
     unsigned int key_lo;
 };
@@ -43,10 +45,12 @@ struct PlanArgs {
     unsigned long long* abits_minmax;  // [BH][2] (scratch)
     SelectTarget* sel;       // [BH][2] (scratch)
     unsigned int* hist;      // [BH][2][4096] (scratch)
+    unsigned int* done_count;  // [BH] finished histogram CTAs of the current pass (scratch)
     uint8_t* prec;           // [BH][R][R]
     int32_t* cnt;            // [2][BH][R]
     uint16_t* kidx;          // [BH][R][R]
     unsigned* status;
+    int num_sms;             // multiprocessors of the device (grid sizing)
 };
 size_t plan_scratch_bytes(int BH, int R);
 void plan_carve_scratch(PlanArgs* p, void* scratch);

@@ -15,6 +15,7 @@
 // of the T8-th and Tkeep-th largest 96-bit keys (A bits : ~pair index), i.e.
 // A descending with ties to the smaller pair index a*R+b, followed by an
 // exact classification and an ordered per-row compaction of the lists.
+#include <algorithm>
 #include <cfloat>
 
 #include "da2_common.cuh"
@@ -268,6 +269,8 @@ __global__ void select_init_kernel(PlanArgs p, long long T8, long long Tk) {
         s.p_lo = 0u;
         s.need = t == 0 ? T8 : Tk;
         s.unique = 0;
+        s.found = 0;
+        s.matches = (long long)p.R * p.R;
         s.none = s.need == 0;
         s.done = s.none;
         s.key_hi = 0ull;
@@ -276,65 +279,32 @@ __global__ void select_init_kernel(PlanArgs p, long long T8, long long Tk) {
     }
 }
 
-constexpr int kHistThreads = 256;
-constexpr int kHistChunk = 16384;
+constexpr int kHistThreads = 1024;
+constexpr int kHistMinChunk = 16384;             // keys per CTA at least (16 per thread)
+constexpr long long kHistDirect = 1ll << 14;     // at most this many matching keys: count in global memory
 
-__global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p) {
-    __shared__ unsigned h[2][4096];
-    const int bh = blockIdx.y;
-    SelectTarget s[2] = {p.sel[bh * 2], p.sel[bh * 2 + 1]};
-    if (s[0].done && s[1].done) return;
-    for (int i = threadIdx.x; i < 2 * 4096; i += kHistThreads) (&h[0][0])[i] = 0u;
-    __syncthreads();
-    unsigned long long mh[2];
-    unsigned ml[2];
-    int w[2], pos[2];
-    for (int t = 0; t < 2; ++t) {
-        top_mask(s[t].nbits, &mh[t], &ml[t]);
-        w[t] = min(12, 96 - s[t].nbits);
-        pos[t] = 96 - s[t].nbits - w[t];
-    }
-    const size_t RR = (size_t)p.R * p.R;
-    const size_t begin = (size_t)blockIdx.x * kHistChunk;
-    const size_t end = min(begin + (size_t)kHistChunk, RR);
-    const double* Ah = p.A + (size_t)bh * RR;
-    for (size_t i = begin + threadIdx.x; i < end; i += kHistThreads) {
-        Key k;
-        k.hi = (unsigned long long)__double_as_longlong(Ah[i]);
-        k.lo = 0xFFFFFFFFu - (unsigned)i;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            if (s[t].done) continue;
-            if (((k.hi ^ s[t].p_hi) & mh[t]) || ((k.lo ^ s[t].p_lo) & ml[t])) continue;
-            if (s[t].unique) {
-                p.sel[bh * 2 + t].key_hi = k.hi;
-                p.sel[bh * 2 + t].key_lo = k.lo;
-                p.sel[bh * 2 + t].done = 1;
-            } else {
-                atomicAdd(&h[t][digit_at(k, pos[t], w[t])], 1u);
-            }
-        }
-    }
-    __syncthreads();
-    unsigned* gh = p.hist + (size_t)bh * 2 * 4096;
-    for (int i = threadIdx.x; i < 2 * 4096; i += kHistThreads) {
-        const unsigned v = (&h[0][0])[i];
-        if (v) atomicAdd(&gh[i], v);
-    }
-}
-
-// One warp per (head, target): choose the digit holding the sought rank.
-__global__ void __launch_bounds__(64) select_scan_kernel(PlanArgs p) {
-    const int bh = blockIdx.x, t = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Choose the digit that holds the sought rank of target t of head bh (one
+// warp), from the completed histogram of the pass, and clear the histogram.
+__device__ void select_scan_warp(PlanArgs& p, int bh, int t, int lane) {
     unsigned* gh = p.hist + ((size_t)bh * 2 + t) * 4096;
     SelectTarget* sp = &p.sel[bh * 2 + t];
-    SelectTarget s = *sp;
-    if (!s.done && !s.unique) {
+    // from L2: another CTA of this pass may have recorded the unique key
+    SelectTarget s;
+    static_assert(sizeof(SelectTarget) % 16 == 0, "SelectTarget is read as 16-byte words");
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(SelectTarget) / 16); ++i)
+        reinterpret_cast<uint4*>(&s)[i] = __ldcg(reinterpret_cast<const uint4*>(sp) + i);
+    if (!s.done && s.unique) {
+        if (s.found) {
+            s.done = 1;
+            if (lane == 0) *sp = s;
+        }
+    } else if (!s.done) {
         const int w = min(12, 96 - s.nbits), pos = 96 - s.nbits - w;
         // lane covers bins [4095 - 128 lane - 127, 4095 - 128 lane], descending
         const int top = 4095 - 128 * lane;
         unsigned long long sum = 0;
-        for (int i = 0; i < 128; ++i) sum += gh[top - i];
+        for (int i = 0; i < 128; ++i) sum += __ldcg(&gh[top - i]);
         unsigned long long incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -347,7 +317,7 @@ __global__ void __launch_bounds__(64) select_scan_kernel(PlanArgs p) {
             long long cum = (long long)excl;
             for (int i = 0; i < 128; ++i) {
                 const int bin = top - i;
-                const long long c = gh[bin];
+                const long long c = __ldcg(&gh[bin]);
                 if (cum + c >= s.need) {
                     s.need -= cum;
                     if (pos >= 32) s.p_hi |= (unsigned long long)bin << (pos - 32);
@@ -356,6 +326,7 @@ __global__ void __launch_bounds__(64) select_scan_kernel(PlanArgs p) {
                         if (pos + w > 32) s.p_hi |= (unsigned long long)bin >> (32 - pos);
                     }
                     s.nbits += w;
+                    s.matches = c;
                     if (s.nbits >= 96) {
                         s.done = 1;
                         s.key_hi = s.p_hi;
@@ -372,6 +343,86 @@ __global__ void __launch_bounds__(64) select_scan_kernel(PlanArgs p) {
     }
     __syncwarp();
     for (int i = lane; i < 4096; i += 32) gh[i] = 0u;
+}
+
+// One pass of the radix selection: histogram of the next digit of the keys
+// that match each target's prefix; the last CTA of a head to finish chooses
+// the digits (select_scan_warp).  A target whose prefix matches one key
+// records that key here and is marked done by that pass's scan, so the
+// `done` flags do not change while a pass runs.
+__global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, int chunk) {
+    __shared__ unsigned h[2][4096];
+    __shared__ int is_last;
+    const int bh = blockIdx.y, tid = threadIdx.x;
+    SelectTarget s[2] = {p.sel[bh * 2], p.sel[bh * 2 + 1]};
+    if (s[0].done && s[1].done) return;
+    bool in_smem[2];
+    for (int t = 0; t < 2; ++t) in_smem[t] = !s[t].done && !s[t].unique && s[t].matches > kHistDirect;
+    if (in_smem[0] || in_smem[1]) {
+        for (int i = tid; i < 2 * 4096; i += kHistThreads) (&h[0][0])[i] = 0u;
+        __syncthreads();
+    }
+    unsigned long long mh[2];
+    unsigned ml[2];
+    int w[2], pos[2];
+    for (int t = 0; t < 2; ++t) {
+        top_mask(s[t].nbits, &mh[t], &ml[t]);
+        w[t] = min(12, 96 - s[t].nbits);
+        pos[t] = 96 - s[t].nbits - w[t];
+    }
+    unsigned* gh = p.hist + (size_t)bh * 2 * 4096;
+    const size_t RR = (size_t)p.R * p.R;
+    const size_t begin = (size_t)blockIdx.x * chunk;
+    const double* Ah = p.A + (size_t)bh * RR;
+    auto count = [&](size_t i, double a) {
+        Key k;
+        k.hi = (unsigned long long)__double_as_longlong(a);
+        k.lo = 0xFFFFFFFFu - (unsigned)i;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (s[t].done) continue;
+            if (((k.hi ^ s[t].p_hi) & mh[t]) || ((k.lo ^ s[t].p_lo) & ml[t])) continue;
+            if (s[t].unique) {
+                p.sel[bh * 2 + t].key_hi = k.hi;
+                p.sel[bh * 2 + t].key_lo = k.lo;
+                p.sel[bh * 2 + t].found = 1;
+            } else if (in_smem[t]) {
+                atomicAdd(&h[t][digit_at(k, pos[t], w[t])], 1u);
+            } else {
+                atomicAdd(&gh[t * 4096 + digit_at(k, pos[t], w[t])], 1u);
+            }
+        }
+    };
+    // chunk / kHistThreads keys per thread (a multiple of 4), four loads in flight
+#pragma unroll 1
+    for (int k0 = 0; k0 < chunk / kHistThreads; k0 += 4) {
+        double a[4];
+        size_t idx[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            idx[u] = begin + (size_t)(k0 + u) * kHistThreads + tid;
+            a[u] = idx[u] < RR ? __ldcs(Ah + idx[u]) : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (idx[u] < RR) count(idx[u], a[u]);
+    }
+    if (in_smem[0] || in_smem[1]) {
+        __syncthreads();
+        for (int i = tid; i < 2 * 4096; i += kHistThreads) {
+            const unsigned v = (&h[0][0])[i];
+            if (v) atomicAdd(&gh[i], v);
+        }
+    }
+    // the last CTA of this head to finish chooses the digits
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(&p.done_count[bh], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (tid < 64) select_scan_warp(p, bh, tid >> 5, tid & 31);
+    if (tid == 0) p.done_count[bh] = 0u;
 }
 
 // ---------------------------------------------------------------- classify
@@ -433,6 +484,8 @@ size_t plan_scratch_bytes(int BH, int R) {
     b += (size_t)2 * BH * sizeof(SelectTarget);
     b = (b + 255) & ~(size_t)255;
     b += (size_t)2 * BH * 4096 * sizeof(unsigned);
+    b = (b + 255) & ~(size_t)255;
+    b += (size_t)BH * sizeof(unsigned);
     return b;
 }
 
@@ -447,6 +500,9 @@ void plan_carve_scratch(PlanArgs* p, void* scratch) {
     off += (size_t)2 * p->BH * sizeof(SelectTarget);
     off = (off + 255) & ~(size_t)255;
     p->hist = reinterpret_cast<unsigned*>(c + off);
+    off += (size_t)2 * p->BH * 4096 * sizeof(unsigned);
+    off = (off + 255) & ~(size_t)255;
+    p->done_count = reinterpret_cast<unsigned*>(c + off);
 }
 
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
@@ -471,6 +527,7 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     if ((e = cudaMemsetAsync(p.abits_minmax, 0xFF, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.abits_minmax + BH, 0, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.hist, 0, sizeof(unsigned) * 2 * 4096 * (size_t)BH, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.done_count, 0, sizeof(unsigned) * (size_t)BH, stream)) != cudaSuccess) return e;
     const size_t smem = sizeof(double) * 2 * R;
     if (smem > 48 * 1024) {
         e = cudaFuncSetAttribute(softmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -479,11 +536,14 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     softmax_kernel<<<(unsigned)((size_t)BH * R), kSoftThreads, smem, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     select_init_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(p, T8, Tk);
-    dim3 hg((unsigned)((RR + kHistChunk - 1) / kHistChunk), BH);
-    for (int pass = 0; pass < kSelectPasses; ++pass) {
-        select_hist_kernel<<<hg, kHistThreads, 0, stream>>>(p);
-        select_scan_kernel<<<BH, 64, 0, stream>>>(p);
-    }
+    // about two 1024-thread CTAs per multiprocessor over all heads, so that
+    // each CTA flushes its shared histogram once for many keys
+    const long long per_head = std::max(1, 2 * std::max(1, p.num_sms) / BH);
+    long long chunk = (RR + per_head - 1) / per_head;
+    chunk = std::max<long long>(kHistMinChunk, (chunk + 4 * kHistThreads - 1) / (4 * kHistThreads) * (4 * kHistThreads));
+    dim3 hg((unsigned)((RR + chunk - 1) / chunk), BH);
+    for (int pass = 0; pass < kSelectPasses; ++pass)
+        select_hist_kernel<<<hg, kHistThreads, 0, stream>>>(p, (int)chunk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     classify_kernel<<<(unsigned)(((size_t)BH * R + 3) / 4), 128, 0, stream>>>(p);
     return cudaGetLastError();

@@ -23,10 +23,20 @@ namespace da2 {
 
 namespace {
 
-constexpr int kThreads = 256;
+// threads per CTA: one quantization item (32 elements of an operand row) per thread
+template <int D>
+constexpr int threads_for() { return D == 64 ? 128 : 256; }
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a K-major
+// no-swizzle operand tile with `row_bytes` bytes per row: core matrices of
+// 8 rows x 16 bytes, adjacent along K, then along the rows.
+__device__ __forceinline__ uint32_t kmajor_offset(int row, int chunk, int row_bytes) {
+    return ((row >> 3) * (row_bytes >> 4) + chunk) * 128 + (row & 7) * 16;
+}
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) prepare_kernel(PrepareArgs p) {
+__global__ void __launch_bounds__(threads_for<D>()) prepare_kernel(PrepareArgs p) {
+    constexpr int kThreads = threads_for<D>();
     constexpr int LD = D + 8;  // padded smem row (bf16 elements) against bank conflicts
     __shared__ __align__(16) uint16_t tile[64 * LD];
     __shared__ int tok[64];
@@ -99,69 +109,100 @@ __global__ void __launch_bounds__(kThreads) prepare_kernel(PrepareArgs p) {
         }
     }
 
-    // Element (row, col) of the operand matrix: Q/K are the tile itself
-    // (rows = slots), V is transposed (rows = channels, cols = slots).
-    const bool vt = (which == 2);
-    const int rows = vt ? D : 64;
-    const int cols = vt ? 64 : D;
-    auto E = [&](int r, int c) -> float { return vt ? X(c, r) : X(r, c); };
-
-    // ---- FP8: cols bytes per row, chunks of 16 in memory order
-    {
-        uint8_t* dst = (which == 0 ? p.q8 : (which == 1 ? p.k8 : p.v8)) + ba * (size_t)(64 * D);
-        const int cpr = cols / 16;
-        for (int m = tid; m < rows * cpr; m += kThreads) {
-            const int grp = m / (8 * cpr), rem = m % (8 * cpr);
-            const int chunk = rem / 8, r = grp * 8 + (rem % 8);
-            uint32_t w[4];
+    // Quantized operand matrices, written in the K-major core-matrix layout:
+    // Q/K rows are the 64 slots (cols = D channels), V^T rows are the D
+    // channels (cols = 64 slots).  Each work item quantizes 32 consecutive
+    // elements of one row to FP8 (two 16-byte chunks) and NVFP4 (one 16-byte
+    // chunk, two scale bytes) from registers.
+    uint8_t* dst8 = (which == 0 ? p.q8 : (which == 1 ? p.k8 : p.v8)) + ba * (size_t)(64 * D);
+    uint8_t* dst4 = (which == 0 ? p.q4 : (which == 1 ? p.k4 : p.v4)) + ba * (size_t)(32 * D);
+    // FP8 e4m3 of 16 values: e4m3(RN(x * inv8)), 0 for a zero tile
+    auto fp8x16 = [&](const float* x) -> uint4 {
+        uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int c = chunk * 16 + e * 4;
-                const uint16_t lo = zero ? 0 : cvt_e4m3x2(__fmul_rn(E(r, c), inv8), __fmul_rn(E(r, c + 1), inv8));
-                const uint16_t hi =
-                    zero ? 0 : cvt_e4m3x2(__fmul_rn(E(r, c + 2), inv8), __fmul_rn(E(r, c + 3), inv8));
-                w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
-            }
-            *reinterpret_cast<uint4*>(dst + (size_t)m * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int e = 0; e < 4; ++e) {
+            const uint16_t lo = zero ? 0 : cvt_e4m3x2(__fmul_rn(x[4 * e], inv8), __fmul_rn(x[4 * e + 1], inv8));
+            const uint16_t hi = zero ? 0 : cvt_e4m3x2(__fmul_rn(x[4 * e + 2], inv8), __fmul_rn(x[4 * e + 3], inv8));
+            w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
         }
-    }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    };
+    // NVFP4 group of 16 values: scale byte sf = e4m3(RN(amax16 * 448/amax)),
+    // codes e2m1(RN(x * RN(1 / RN(value(sf) * g4)))) into 8 bytes
+    auto fp4x16 = [&](const float* x, uint8_t* sf_out) -> uint2 {
+        float a16 = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) a16 = fmaxf(a16, fabsf(x[e]));
+        const uint32_t sf = zero ? 0u : (uint32_t)(cvt_e4m3x2(__fmul_rn(a16, t4), 0.0f) & 0xFF);
+        *sf_out = (uint8_t)sf;
+        if (sf == 0) return make_uint2(0u, 0u);
+        const float rcp = __frcp_rn(__fmul_rn(e4m3_to_f32((uint8_t)sf), g4));
+        uint32_t w[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc |= (uint32_t)cvt_e2m1x2(__fmul_rn(x[8 * h + 2 * e], rcp), __fmul_rn(x[8 * h + 2 * e + 1], rcp))
+                       << (8 * e);
+            w[h] = acc;
+        }
+        return make_uint2(w[0], w[1]);
+    };
+    auto bf_lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+    auto bf_hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
 
-    // ---- NVFP4: cols/2 bytes per row; one 16-byte chunk = 32 elements = 2 groups
-    {
-        uint8_t* dst = (which == 0 ? p.q4 : (which == 1 ? p.k4 : p.v4)) + ba * (size_t)(32 * D);
-        const int cpr = cols / 32;
-        for (int m = tid; m < rows * cpr; m += kThreads) {
-            const int grp = m / (8 * cpr), rem = m % (8 * cpr);
-            const int chunk = rem / 8, r = grp * 8 + (rem % 8);
-            uint8_t bytes[16];
+    if (which < 2) {
+        // item (slot r, 32-channel chunk k); a warp covers 32 consecutive slots
+        // of one chunk: its 16-byte shared reads fall in distinct banks
+        for (int it = tid; it < 64 * (D / 32); it += kThreads) {
+            const int r = it & 63, k = it >> 6;
+            float x[32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = *reinterpret_cast<const uint4*>(&tile[r * LD + 32 * k + 8 * q]);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x[8 * q + 2 * e] = bf_lo(ww[e]);
+                    x[8 * q + 2 * e + 1] = bf_hi(ww[e]);
+                }
+            }
+            *reinterpret_cast<uint4*>(dst8 + kmajor_offset(r, 2 * k, D)) = fp8x16(x);
+            *reinterpret_cast<uint4*>(dst8 + kmajor_offset(r, 2 * k + 1, D)) = fp8x16(x + 16);
+            uint8_t sf0, sf1;
+            const uint2 c0 = fp4x16(x, &sf0), c1 = fp4x16(x + 16, &sf1);
+            *reinterpret_cast<uint4*>(dst4 + kmajor_offset(r, k, D / 2)) = make_uint4(c0.x, c0.y, c1.x, c1.y);
 #pragma unroll
             for (int gi = 0; gi < 2; ++gi) {
-                const int c0 = chunk * 32 + gi * 16;
-                float v[16], a16 = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    v[e] = E(r, c0 + e);
-                    a16 = fmaxf(a16, fabsf(v[e]));
-                }
-                uint8_t sf = 0;
-                if (!zero) sf = (uint8_t)(cvt_e4m3x2(__fmul_rn(a16, t4), 0.0f) & 0xFF);
-                const float rcp = sf ? __fdiv_rn(1.0f, __fmul_rn(e4m3_to_f32(sf), g4)) : 0.0f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    bytes[gi * 8 + e] = sf ? cvt_e2m1x2(__fmul_rn(v[2 * e], rcp), __fmul_rn(v[2 * e + 1], rcp)) : 0;
-                // scale byte: group index along the row is c0/16
-                const int gcol = c0 / 16;
-                if (which == 0) {
-                    sf_atom[r * (D / 16) + gcol] = sf;
-                } else if (which == 1) {
-                    sf_atom[16 * (r & 31) + 4 * (2 * (c0 / 64) + (r >> 5)) + (c0 % 64) / 16] = sf;
-                } else {
-                    sf_atom[16 * (r & 31) + 4 * (r >> 5) + gcol] = sf;
-                }
+                const int gcol = 2 * k + gi;  // group index along the row
+                const uint8_t sf = gi ? sf1 : sf0;
+                if (which == 0) sf_atom[r * (D / 16) + gcol] = sf;
+                else sf_atom[16 * (r & 31) + 4 * (2 * (gcol / 4) + (r >> 5)) + (gcol % 4)] = sf;
             }
-            uint4 out;
-            memcpy(&out, bytes, 16);
-            *reinterpret_cast<uint4*>(dst + (size_t)m * 16) = out;
+        }
+    } else {
+        // V^T: item (channel pair 2c, 2c+1; 16-slot group k); one 32-bit shared
+        // read gives both channels of a slot, a warp reads 128 contiguous bytes
+        for (int it = tid; it < (D / 2) * 4; it += kThreads) {
+            const int c = it % (D / 2), k = it / (D / 2);
+            float x0[16], x1[16];
+#pragma unroll
+            for (int sl = 0; sl < 16; ++sl) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(&tile[(16 * k + sl) * LD + 2 * c]);
+                x0[sl] = bf_lo(w);
+                x1[sl] = bf_hi(w);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = 2 * c + h;
+                const float* x = h ? x1 : x0;
+                *reinterpret_cast<uint4*>(dst8 + kmajor_offset(row, k, 64)) = fp8x16(x);
+                uint8_t sf;
+                const uint2 c4 = fp4x16(x, &sf);
+                *reinterpret_cast<uint2*>(dst4 + kmajor_offset(row, k >> 1, 32) + 8 * (k & 1)) = c4;
+                sf_atom[16 * (row & 31) + 4 * (row >> 5) + k] = sf;
+            }
         }
     }
     __syncthreads();
@@ -188,8 +229,8 @@ cudaError_t launch_prepare(const PrepareArgs& p, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(p.vmax, 0, sizeof(float) * 2 * BH, stream);
     if (e != cudaSuccess) return e;
     dim3 grid(p.R, BH, 3);
-    if (p.d == 64) prepare_kernel<64><<<grid, kThreads, 0, stream>>>(p);
-    else prepare_kernel<128><<<grid, kThreads, 0, stream>>>(p);
+    if (p.d == 64) prepare_kernel<64><<<grid, threads_for<64>(), 0, stream>>>(p);
+    else prepare_kernel<128><<<grid, threads_for<128>(), 0, stream>>>(p);
     return cudaGetLastError();
 }
 
