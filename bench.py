@@ -186,22 +186,52 @@ def run_ours(args, w, rank, world):
         per["plan"].append(e[1].elapsed_time(e[2]))
         per["attention"].append(e[2].elapsed_time(e[3]))
 
-    # ---- end to end through the C ABI with host buffers
+    # ---- end to end through the C ABI with host buffers, pipelined over steps:
+    # step i uploads its inputs (pinned host -> device) on an upload stream,
+    # runs prepare + plan + attention on the compute stream and downloads its
+    # output on a download stream; two device buffer sets let the upload of
+    # step i+1 and the download of step i-1 overlap the compute of step i.
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    bufs = [(q, k, v, out)] + [tuple(torch.empty_like(t) for t in (q, k, v, out))]
+    outs_h = [out_h, torch.empty_like(out_h).pin_memory()]
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            q.copy_(qh, non_blocking=True)
-            k.copy_(kh, non_blocking=True)
-            v.copy_(vh, non_blocking=True)
-            step()
-            out_h.copy_(out, non_blocking=True)
-    e1.record(stream)
-    stream.synchronize()
+    e0.record(up)
+    for i in range(args.steps):
+        j = i & 1
+        qb, kb, vb, ob = bufs[j]
+        if i >= 2:
+            up.wait_event(ev_comp[j])  # the compute of step i-2 has read buffer set j
+        with torch.cuda.stream(up):
+            qb.copy_(qh, non_blocking=True)
+            kb.copy_(kh, non_blocking=True)
+            vb.copy_(vh, non_blocking=True)
+        ev_up[j].record(up)
+        stream.wait_event(ev_up[j])
+        if i >= 2:
+            stream.wait_event(ev_down[j])  # the output of step i-2 has left buffer set j
+        with torch.cuda.stream(stream):
+            m.prepare(qb, kb, vb, prep, stream)
+            m.plan(prep, plan, w.bp8, w.bp4, w.lam, stream)
+            m.attention(prep, plan, ob, stream)
+        ev_comp[j].record(stream)
+        down.wait_event(ev_comp[j])
+        with torch.cuda.stream(down):
+            outs_h[j].copy_(ob, non_blocking=True)
+        ev_down[j].record(down)
+    up.wait_event(ev_down[(args.steps - 1) & 1])
+    if args.steps >= 2:
+        up.wait_event(ev_down[(args.steps - 2) & 1])
+    e1.record(up)
+    up.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    torch.cuda.synchronize(dev)
+    m.check_status(stream)
     barrier()
 
     vals = torch.tensor([total_ms, e2e_ms] + [sum(per[k]) for k in ("prepare", "plan", "attention")],
@@ -343,7 +373,9 @@ def main():
         "clocks": r["clocks"],
         "e2e": {"value": world * flops / (r["e2e_ms"] / args.steps * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                "ms_per_step": r["e2e_ms"] / args.steps},
+                "ms_per_step": r["e2e_ms"] / args.steps,
+                "schedule": "pinned host buffers; upload, compute and download streams pipelined over steps "
+                            "(two device buffer sets)"},
         "gpu_launches": launches_per_step * args.steps,
     }
     # prepare: algorithmic bytes = bf16 Q/K/V read + every prepared output written once
