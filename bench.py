@@ -120,6 +120,15 @@ def kept_pair_counts(plan_cnt, B, H, R):
     return int(c[0].sum().item()), int(c[1].sum().item())
 
 
+def max_over_ranks(vals, world: int):
+    """Element-wise maximum of a timing vector over all ranks (the job's time
+    is its slowest rank's); identity on one rank."""
+    import torch
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    return vals
+
+
 def run_ours(args, w, rank, world):
     import torch
 
@@ -236,9 +245,7 @@ def run_ours(args, w, rank, world):
 
     vals = torch.tensor([total_ms, e2e_ms] + [sum(per[k]) for k in ("prepare", "plan", "attention")],
                         dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms, t_prep, t_plan, t_attn = vals.tolist()
+    total_ms, e2e_ms, t_prep, t_plan, t_attn = max_over_ranks(vals, world).tolist()
     m.close()
     return dict(total_ms=total_ms, e2e_ms=e2e_ms, t_prep=t_prep / args.steps, t_plan=t_plan / args.steps,
                 t_attn=t_attn / args.steps, n8=n8, n4=n4, R=m.R, clocks=clk,
