@@ -25,15 +25,13 @@
 //              winning key is exactly 1), rescales its row of O when m grows
 //              and once at the phase switch (sigma8 -> sigma4, the change of
 //              units of Eq. 8), and in the epilogue divides by l, converts to
-//              bf16 and stores the row at its original token position.  The
-//              template also builds a two-threads-per-row split (RT = 2: 8
-//              softmax warps, each owning 32 of the 64 columns, the pair
-//              exchanging its partial row max through shared memory).
-//   warp 4RT   MMA issue (one thread): S = Q K^T (tcgen05.mma kind::f8f6f4 or
-//              kind::mxf4nvf4 block16) into the S buffer, O += P V into the
-//              single O accumulator.
-//   warp 4RT+1 loader (one thread): bulk async copies of the K / V tiles
-//              (pre-tiled by the preparation kernel) into a 3-stage ring.
+//              bf16 and stores the row at its original token position.
+//   warp 4     MMA issue (whole warp, one elected lane issues): S = Q K^T
+//              (tcgen05.mma kind::f8f6f4 or kind::mxf4nvf4 block16) into the S
+//              buffer, O += P V into the single O accumulator.
+//   warp 5     loader (whole warp, one elected lane issues): bulk async copies
+//              of the K / V tiles (pre-tiled by the preparation kernel) into a
+//              3-stage ring, and the step record of each stage.
 // Every mbarrier wait is bounded; a stuck wait sets the status word, all
 // roles drain their own outstanding work and the CTA frees tensor memory
 // before returning.
@@ -45,24 +43,13 @@ namespace da2 {
 namespace {
 
 constexpr int kStages = 3;
-// Of every 8 exponential pairs of a 16-key group, this many are computed on
-// the FMA pipe (exp2_poly) instead of the MUFU unit.
-#ifndef DA2_POLY_PAIRS
-#define DA2_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = DA2_POLY_PAIRS;
-// Softmax threads per row of the tile (1: each thread owns all 64 key columns
-// of a step; 2: two threads split them and exchange the partial row max).
-constexpr int kRowThreads = 1;
-
-template <int RT>
-struct Cfg {
-    static constexpr int kSoftThreads = 128 * RT;
-    static constexpr int kThreads = kSoftThreads + 64;
-    static constexpr int kMmaWarp = 4 * RT, kLoadWarp = 4 * RT + 1;
-    static constexpr int CW = 64 / RT;  // key columns per softmax thread
-    static constexpr int NP = CW / 2;   // float2 pairs per softmax thread
-};
+// Roles: softmax warps 0-3 (one thread per tile row, all 64 key columns of a
+// step), MMA warp 4, loader warp 5.
+constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = kSoftmaxThreads + 64;
+constexpr int kMmaWarp = 4, kLoadWarp = 5;
+constexpr int CW = 64;      // key columns per softmax thread
+constexpr int NP = CW / 2;  // float2 pairs per softmax thread
 constexpr uint32_t kTmemCols = 256;
 // tensor-memory column map (per CTA)
 constexpr uint32_t kColO = 0;      // O accumulator, D columns
@@ -94,8 +81,7 @@ struct Smem {
     static constexpr uint32_t p = stage + kStages * stage_bytes;  // 2 x (128 x 64 + 512)
     static constexpr uint32_t p_bytes = 128 * 64 + 512;
     static constexpr uint32_t bitmap = p + 2 * p_bytes;        // 4 x 128 words
-    static constexpr uint32_t xmax = bitmap + 4 * 128 * 4;     // [2 steps][2 halves][128 rows] floats
-    static constexpr uint32_t rcp = xmax + 2 * 2 * 128 * 4;    // 128 floats: 1/value of each ue4m3 code
+    static constexpr uint32_t rcp = bitmap + 4 * 128 * 4;      // 128 floats: 1/value of each ue4m3 code
     static constexpr uint32_t meta = rcp + 128 * 4;            // kStages x 32 copies of the StepMeta record
     static constexpr uint32_t list = meta + kStages * 512;     // 2R entries of 16 bits
 };
@@ -121,25 +107,6 @@ __device__ __forceinline__ float div6(float x) {
     return fmaf(r, c, q);
 }
 
-// 32 consecutive fp32 columns of this warp's tensor-memory lanes into
-// v[O..O+15] as pairs; load and wait in one asm statement (see tmem_ld32).
-template <int O, int NP>
-__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr, float2 (&v)[NP]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=f"(v[O + 0].x), "=f"(v[O + 0].y), "=f"(v[O + 1].x), "=f"(v[O + 1].y), "=f"(v[O + 2].x),
-          "=f"(v[O + 2].y), "=f"(v[O + 3].x), "=f"(v[O + 3].y), "=f"(v[O + 4].x), "=f"(v[O + 4].y),
-          "=f"(v[O + 5].x), "=f"(v[O + 5].y), "=f"(v[O + 6].x), "=f"(v[O + 6].y), "=f"(v[O + 7].x),
-          "=f"(v[O + 7].y), "=f"(v[O + 8].x), "=f"(v[O + 8].y), "=f"(v[O + 9].x), "=f"(v[O + 9].y),
-          "=f"(v[O + 10].x), "=f"(v[O + 10].y), "=f"(v[O + 11].x), "=f"(v[O + 11].y), "=f"(v[O + 12].x),
-          "=f"(v[O + 12].y), "=f"(v[O + 13].x), "=f"(v[O + 13].y), "=f"(v[O + 14].x), "=f"(v[O + 14].y),
-          "=f"(v[O + 15].x), "=f"(v[O + 15].y)
-        : "r"(taddr)
-        : "memory");
-}
-
 // 64 consecutive fp32 columns of this warp's tensor-memory lanes into v[0..31]
 // as pairs, and 4 columns of the step record into r: two loads and one wait
 // in one asm statement.
@@ -152,30 +119,6 @@ __device__ __forceinline__ void tmem_ld64x2_rec(uint32_t taddr, uint32_t raddr, 
         : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x), "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y), "=f"(v[7].x), "=f"(v[7].y), "=f"(v[8].x), "=f"(v[8].y), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[10].x), "=f"(v[10].y), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[13].x), "=f"(v[13].y), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[15].x), "=f"(v[15].y), "=f"(v[16].x), "=f"(v[16].y), "=f"(v[17].x), "=f"(v[17].y), "=f"(v[18].x), "=f"(v[18].y), "=f"(v[19].x), "=f"(v[19].y), "=f"(v[20].x), "=f"(v[20].y), "=f"(v[21].x), "=f"(v[21].y), "=f"(v[22].x), "=f"(v[22].y), "=f"(v[23].x), "=f"(v[23].y), "=f"(v[24].x), "=f"(v[24].y), "=f"(v[25].x), "=f"(v[25].y), "=f"(v[26].x), "=f"(v[26].y), "=f"(v[27].x), "=f"(v[27].y), "=f"(v[28].x), "=f"(v[28].y), "=f"(v[29].x), "=f"(v[29].y), "=f"(v[30].x), "=f"(v[30].y), "=f"(v[31].x), "=f"(v[31].y),
           "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
         : "r"(taddr), "r"(raddr)
-        : "memory");
-}
-
-// 32 consecutive fp32 columns into v[0..15] as pairs and the 4 columns of the
-// step record into r (two loads, one wait).
-[[maybe_unused]] __device__ __forceinline__ void tmem_ld32x2_rec(uint32_t taddr, uint32_t raddr, float2 (&v)[16],
-                                                uint32_t (&r)[4]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%36];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%32,%33,%34,%35}, [%37];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=f"(v[0].x), "=f"(v[0].y), "=f"(v[1].x), "=f"(v[1].y), "=f"(v[2].x), "=f"(v[2].y), "=f"(v[3].x), "=f"(v[3].y), "=f"(v[4].x), "=f"(v[4].y), "=f"(v[5].x), "=f"(v[5].y), "=f"(v[6].x), "=f"(v[6].y), "=f"(v[7].x), "=f"(v[7].y), "=f"(v[8].x), "=f"(v[8].y), "=f"(v[9].x), "=f"(v[9].y), "=f"(v[10].x), "=f"(v[10].y), "=f"(v[11].x), "=f"(v[11].y), "=f"(v[12].x), "=f"(v[12].y), "=f"(v[13].x), "=f"(v[13].y), "=f"(v[14].x), "=f"(v[14].y), "=f"(v[15].x), "=f"(v[15].y),
-          "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-        : "r"(taddr), "r"(raddr)
-        : "memory");
-}
-
-// 4 consecutive 32-bit columns of this warp's tensor-memory lanes (load and wait).
-[[maybe_unused]] __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-        : "r"(taddr)
         : "memory");
 }
 
@@ -193,31 +136,6 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
                  :
                  : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
                  : "memory");
-}
-
-// 2^t (t <= 0, or -inf) for two values on the FMA pipe, an alternative to
-// the MUFU ex2 for part of the weights.  t is clamped to -126 (results stay
-// normal; 2^-126 is far below the smallest weight code), split as n + f with
-// n = round(t) (added to 1.5 * 2^23, whose low mantissa bits then hold n) and
-// f in [-1/2, 1/2]; 2^f = 1 + f * q(f) with q of degree 4 fitted to relative
-// error 2e-7 on that interval (the constant term 1 gives 2^0 = 1 exactly);
-// 2^n is applied by adding n to the exponent field.
-__device__ __forceinline__ float2 exp2_poly(float2 t) {
-    t.x = fmaxf(t.x, -126.0f);
-    t.y = fmaxf(t.y, -126.0f);
-    const float2 big = make_float2(12582912.0f, 12582912.0f);
-    const float2 r = __fadd2_rn(t, big);
-    const float2 n = __fadd2_rn(r, make_float2(-12582912.0f, -12582912.0f));
-    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), t);
-    float2 q = __ffma2_rn(make_float2(1.3264722656e-3f, 1.3264722656e-3f), f,
-                          make_float2(9.6715129912e-3f, 9.6715129912e-3f));
-    q = __ffma2_rn(q, f, make_float2(5.5507335812e-2f, 5.5507335812e-2f));
-    q = __ffma2_rn(q, f, make_float2(2.4022242427e-1f, 2.4022242427e-1f));
-    q = __ffma2_rn(q, f, make_float2(6.9314700365e-1f, 6.9314700365e-1f));
-    float2 p = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
-    p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(r.x) << 23));
-    p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(r.y) << 23));
-    return p;
 }
 
 // Four fp32 -> four e4m3 bytes in one word (first value in the low byte).
@@ -246,43 +164,6 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(float2 a, float2 b, float2 c, fl
     return w;
 }
 
-// Max over the 2*NP values of the pairs v[0..NP) (NP = 16 or 32): a tree of
-// 3-input maxima (all indices are compile-time after unrolling).
-template <int NP>
-__device__ __forceinline__ float pair_val(const float2 (&v)[NP], int k) {
-    return (k & 1) ? v[k >> 1].y : v[k >> 1].x;
-}
-template <int NP>
-__device__ __forceinline__ float rowmax_pairs(const float2 (&v)[NP]) {
-    constexpr int n0 = 2 * NP, n1 = (n0 + 2) / 3;
-    float t[n1];
-#pragma unroll
-    for (int i = 0; i < n1; ++i) {
-        const int k = 3 * i;
-        const float a = pair_val<NP>(v, k);
-        const float b = k + 1 < n0 ? pair_val<NP>(v, k + 1) : a;
-        const float c = k + 2 < n0 ? pair_val<NP>(v, k + 2) : a;
-        t[i] = max3f(a, b, c);
-    }
-    int n = n1;
-#pragma unroll
-    for (int round = 0; round < 4; ++round) {
-        if (n > 1) {
-#pragma unroll
-            for (int i = 0; i < (n1 + 2) / 3; ++i) {
-                if (3 * i < n) {
-                    const float a = t[3 * i];
-                    const float b = 3 * i + 1 < n ? t[3 * i + 1] : a;
-                    const float c = 3 * i + 2 < n ? t[3 * i + 2] : a;
-                    t[i] = max3f(a, b, c);
-                }
-            }
-            n = (n + 2) / 3;
-        }
-    }
-    return t[0];
-}
-
 // Max of the 16 consecutive values v[b..b+7] (pairs).
 template <int NP>
 __device__ __forceinline__ float groupmax16_raw(const float2 (&v)[NP], int b) {
@@ -292,28 +173,16 @@ __device__ __forceinline__ float groupmax16_raw(const float2 (&v)[NP], int b) {
     return max3f(max3f(t0, t1, t2), t3, fmaxf(t4, v[b + 7].y));
 }
 
-// Max of 16 consecutive values v[b..b+7] (pairs) and 0.
-template <int NP>
-__device__ __forceinline__ float groupmax16(const float2 (&v)[NP], int b) {
-    const float t0 = max3f(v[b].x, v[b].y, v[b + 1].x), t1 = max3f(v[b + 1].y, v[b + 2].x, v[b + 2].y);
-    const float t2 = max3f(v[b + 3].x, v[b + 3].y, v[b + 4].x), t3 = max3f(v[b + 4].y, v[b + 5].x, v[b + 5].y);
-    const float t4 = max3f(v[b + 6].x, v[b + 6].y, v[b + 7].x);
-    return max3f(max3f(t0, t1, t2), max3f(t3, t4, v[b + 7].y), 0.0f);
-}
 
-template <int D, int RT>
-__global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArgs p) {
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
     using L = Smem<D>;
-    using C = Cfg<RT>;
-    constexpr int kThreads = C::kThreads, kSoftmaxThreads = C::kSoftThreads;
-    constexpr int kMmaWarp = C::kMmaWarp, kLoadWarp = C::kLoadWarp;
-    constexpr int CW = C::CW, NP = C::NP;
     extern __shared__ __align__(1024) uint8_t smem[];
     // bar_empty[st] completes when the PV of a step in stage st has finished:
     // it frees the stage for the loader and tells the softmax threads that O
     // holds that step
     __shared__ uint64_t bar_q, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
-        bar_x[4], bar_drain;
+        bar_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh, item_sh;
     __shared__ int n_ent_sh[2];
@@ -342,7 +211,6 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar_p[s], kSoftmaxThreads / 32);
         }
-        for (int s = 0; s < 4; ++s) mbar_init(&bar_x[s], 64);  // the two warps of a row quarter
         mbar_init(&bar_drain, 1);
         abort_sh = 0;
         fence_mbar_init();
@@ -363,7 +231,6 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
     uint32_t gstep = 0;         // steps processed by this CTA before the current item
     uint32_t nitem = 0;         // items processed by this CTA
     uint32_t loads_issued = 0;  // loader: stage fills issued (for the final drain)
-    uint32_t nx = 0;            // softmax: exchanges with the partner warp so far
     bool mma_issued = false;
 
     for (;;) {
@@ -558,7 +425,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             if (ok && n_ent > 0) wait_all(&bar_sfree, (gstep + n_ent - 1) & 1);
         } else {
             // ================================================== softmax
-            const int quarter = warp & 3, hh = warp >> 2;  // lane quarter, column share (0 when RT == 1)
+            const int quarter = warp;                       // tensor-memory lane quarter
             const int r = 32 * quarter + lane;              // tile row
             const int hf = quarter >> 1;                    // which query block of the pair (= r >> 6)
             const int a = hf ? a1 : a0;
@@ -566,10 +433,9 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
             const size_t ta = (size_t)bh * R + (qvalid ? a : a0);
             const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
             const float rdl2e = (D == 64 ? 0.125f : 0.0883883461356163025f) * 1.4426950408889634f;
-            float* xmax = reinterpret_cast<float*>(smem + L::xmax);
             const float* rcp_tab = reinterpret_cast<const float*>(smem + L::rcp);
             // Q scale factors of this row into the copy atoms (one per 64 channels)
-            for (int ch = hh; ch < D / 64; ch += RT) {
+            for (int ch = 0; ch < D / 64; ++ch) {
                 uint8_t* atom = smem + L::sfq;
                 const uint8_t* src = p.sfq + ta * (64 * (D / 16)) + (r & 63) * (D / 16);
                 const uint32_t w = qvalid ? *reinterpret_cast<const uint32_t*>(src + 4 * ch) : 0u;
@@ -602,26 +468,9 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 tc_fence_after();
                 float2 v[NP];
                 StepMeta mt;
-                float pmax_raw = -INFINITY;  // RT == 2: raw maximum of the partner's columns
                 if (active) {
                     uint32_t mw[4];
-                    if constexpr (CW == 64) {
-                        tmem_ld64x2_rec(lane_base + kColS, lane_base + kColMeta, v, mw);
-                    } else {
-                        // the partner warp's columns first, for the row maximum
-                        // only (no exchange between the two warps of a row)
-                        tmem_ld32x2_rec(lane_base + kColS + CW * (1 - hh), lane_base + kColMeta, v, mw);
-                        const int nkp = (int)mw[0] - CW * (1 - hh);
-                        if (nkp < CW) {
-#pragma unroll
-                            for (int i = 0; i < NP; ++i) {
-                                if (2 * i >= nkp) v[i].x = -INFINITY;
-                                if (2 * i + 1 >= nkp) v[i].y = -INFINITY;
-                            }
-                        }
-                        pmax_raw = rowmax_pairs<NP>(v);
-                        tmem_ld32x2<0>(lane_base + kColS + CW * hh, v);
-                    }
+                    tmem_ld64x2_rec(lane_base + kColS, lane_base + kColMeta, v, mw);
                     mt.nk = (int)mw[0];
                     mt.ck = __uint_as_float(mw[1]);
                     mt.ratio = __uint_as_float(mw[2]);
@@ -643,7 +492,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     const float2 c22 = make_float2(c2, c2);
 #pragma unroll
                     for (int i = 0; i < NP; ++i) v[i] = __fmul2_rn(v[i], c22);
-                    const int nk = mt.nk - CW * hh;  // valid keys among this thread's columns
+                    const int nk = mt.nk;  // valid keys of the block
                     if (nk < CW) {
                         if (nk >= CW - 16) {
 #pragma unroll
@@ -669,13 +518,6 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
 #pragma unroll
                     for (int gi = 1; gi < NGR; gi += 2)
                         rmx = gi + 1 < NGR ? max3f(rmx, gm[gi], gm[gi + 1]) : fmaxf(rmx, gm[gi]);
-                    if (RT == 2) {
-                        // The partner scales its columns by the same c2 and
-                        // rounding is monotonic, so the maximum of its scaled
-                        // values is the scaled raw maximum: both warps of the
-                        // row get the same row maximum bit for bit.
-                        if (pmax_raw != -INFINITY) rmx = fmaxf(rmx, pmax_raw * c2);
-                    }
                     const float mn = fmaxf(m, rmx);
                     if (m != -INFINITY && mn > m) {
                         corr = ex2f(m - mn);
@@ -690,8 +532,8 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
 #pragma unroll
                         for (int i = b; i < b + 8; i += 2) {
                             const float2 t0 = __fadd2_rn(v[i], nm), t1 = __fadd2_rn(v[i + 1], nm);
-                            const float2 p0 = ((i - b) < kPolyPairs) ? exp2_poly(t0) : make_float2(ex2f(t0.x), ex2f(t0.y));
-                            const float2 p1 = ((i + 1 - b) < kPolyPairs) ? exp2_poly(t1) : make_float2(ex2f(t1.x), ex2f(t1.y));
+                            const float2 p0 = make_float2(ex2f(t0.x), ex2f(t0.y));
+                            const float2 p1 = make_float2(ex2f(t1.x), ex2f(t1.y));
                             acc0 = __fadd2_rn(acc0, p0);
                             acc1 = __fadd2_rn(acc1, p1);
                             v[i] = __fmul2_rn(p0, rt);
@@ -706,7 +548,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                         for (int ch = 0; ch < CW / 16; ++ch) {
                             const int b = ch * 8;
                             exp_group(b);
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 16) * hh + ch, 64)) =
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) =
                                 make_uint4(pack_e4m3x4(v[b], v[b + 1]), pack_e4m3x4(v[b + 2], v[b + 3]),
                                            pack_e4m3x4(v[b + 4], v[b + 5]), pack_e4m3x4(v[b + 6], v[b + 7]));
                         }
@@ -735,7 +577,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
 #pragma unroll
                             for (int i = 0; i < 8; ++i) {
                                 const float2 tt = __fadd2_rn(v[8 * gi + i], nm);
-                                const float2 pp = i < kPolyPairs ? exp2_poly(tt) : make_float2(ex2f(tt.x), ex2f(tt.y));
+                                const float2 pp = make_float2(ex2f(tt.x), ex2f(tt.y));
                                 if (i & 1) acc1 = __fadd2_rn(acc1, pp);
                                 else acc0 = __fadd2_rn(acc0, pp);
                                 y[i] = __fmul2_rn(pp, sg2);
@@ -746,11 +588,10 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                         // 32 keys = one 16-byte chunk of the 32-byte row
 #pragma unroll
                         for (int ch = 0; ch < CW / 32; ++ch)
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 32) * hh + ch, 32)) =
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 32)) =
                                 make_uint4(wq[4 * ch], wq[4 * ch + 1], wq[4 * ch + 2], wq[4 * ch + 3]);
                         uint8_t* sfp = pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5);
-                        if (RT == 1) *reinterpret_cast<uint32_t*>(sfp) = sfw;
-                        else *reinterpret_cast<uint16_t*>(sfp + 2 * hh) = (uint16_t)sfw;
+                        *reinterpret_cast<uint32_t*>(sfp) = sfw;
                     }
                     const float2 a2 = __fadd2_rn(acc0, acc1);
                     l = l * corr + (a2.x + a2.y);
@@ -759,16 +600,15 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     if (ph == 0) {
 #pragma unroll
                         for (int ch = 0; ch < CW / 16; ++ch)
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 16) * hh + ch, 64)) =
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 64)) =
                                 make_uint4(0, 0, 0, 0);
                     } else {
 #pragma unroll
                         for (int ch = 0; ch < CW / 32; ++ch)
-                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, (CW / 32) * hh + ch, 32)) =
+                            *reinterpret_cast<uint4*>(pbuf + kmajor_off(r, ch, 32)) =
                                 make_uint4(0, 0, 0, 0);
                         uint8_t* sfp = pbuf + 128 * 64 + 16 * (r & 31) + 4 * (r >> 5);
-                        if (RT == 1) *reinterpret_cast<uint32_t*>(sfp) = 0u;
-                        else *reinterpret_cast<uint16_t*>(sfp + 2 * hh) = 0;
+                        *reinterpret_cast<uint32_t*>(sfp) = 0u;
                     }
                 }
                 // O rescale (this thread's half of the columns): when the row
@@ -784,30 +624,18 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                     if (ok) {
                         tc_fence_after();
                         const uint64_t f2 = need ? pack2(f, f) : pack2(1.0f, 1.0f);
-                        // this thread's D/RT columns of O, in 64-column round trips
-                        // (32 when it owns only 32)
-                        constexpr int OW = (RT == 1 && (D / RT) % 64 == 0) ? 64 : 32;
+                        // this thread's row of O, in 64-column round trips
 #pragma unroll 1
-                        for (int c0 = hh * (D / RT); c0 < (hh + 1) * (D / RT); c0 += OW) {
+                        for (int c0 = 0; c0 < D; c0 += 64) {
                             uint32_t o[64];
-                            if constexpr (OW == 64) {
-                                tmem_ld64(lane_base + kColO + c0, o);
-                            } else {
-                                uint32_t (&o32)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
-                                tmem_ld32(lane_base + kColO + c0, o32);
-                            }
+                            tmem_ld64(lane_base + kColO + c0, o);
 #pragma unroll
-                            for (int c = 0; c < OW; c += 2) {
+                            for (int c = 0; c < 64; c += 2) {
                                 const uint64_t v = mul2(pack2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), f2);
                                 o[c] = __float_as_uint(lo2(v));
                                 o[c + 1] = __float_as_uint(hi2(v));
                             }
-                            if constexpr (OW == 64) {
-                                tmem_st64(lane_base + kColO + c0, o);
-                            } else {
-                                const uint32_t (&o32)[32] = *reinterpret_cast<const uint32_t(*)[32]>(&o[0]);
-                                tmem_st32(lane_base + kColO + c0, o32);
-                            }
+                            tmem_st64(lane_base + kColO + c0, o);
                         }
                         tc_wait_st();
                     }
@@ -819,18 +647,9 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_p[pb]);
             }
-            // ---- epilogue: both halves of the denominator, then this thread's columns
+            // ---- epilogue: O / l, bf16, stored at the row's token
             ok = __all_sync(0xffffffffu, ok);
-            float lt = l;
-            if (RT == 2) {
-                float* xl = xmax + (nx & 1) * 256;
-                xl[hh * 128 + r] = l;
-                mbar_arrive(&bar_x[quarter]);
-                const bool xw = mbar_wait(&bar_x[quarter], nx & 1, abort_v, p.status);
-                ++nx;
-                if (!__all_sync(0xffffffffu, xw)) ok = false;
-                lt = xl[r] + xl[128 + r];
-            }
+            const float lt = l;
             float o_scale = 0.0f;
             const bool have = n_ent > 0 && ok;
             if (have) {
@@ -849,7 +668,7 @@ __global__ void __launch_bounds__(Cfg<RT>::kThreads, 2) attention_kernel(AttnArg
                 dst += (size_t)(bh / p.H) * p.o0 + (size_t)(bh % p.H) * p.o1 + (size_t)t * p.o2;
             }
 #pragma unroll 1
-            for (int c0 = hh * (D / RT); c0 < (hh + 1) * (D / RT); c0 += 32) {
+            for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
                 if (have_o) {
                     tmem_ld32(lane_base + kColO + c0, o);
@@ -911,20 +730,19 @@ cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream) {
     const int items = p.B * p.H * ((p.R + 1) / 2);
     if (items == 0) return cudaSuccess;
     const int grid = items < 2 * p.num_sms ? items : 2 * p.num_sms;
-    constexpr int RT = kRowThreads;
-    constexpr int threads = Cfg<RT>::kThreads;
+    constexpr int threads = kThreads;
     cudaError_t e = cudaMemsetAsync(p.work_counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
     if (p.d == 64) {
         const size_t smem = attention_smem_bytes<64>(p.R);
-        e = cudaFuncSetAttribute(attention_kernel<64, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(attention_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attention_kernel<64, RT><<<grid, threads, smem, stream>>>(p);
+        attention_kernel<64><<<grid, threads, smem, stream>>>(p);
     } else {
         const size_t smem = attention_smem_bytes<128>(p.R);
-        e = cudaFuncSetAttribute(attention_kernel<128, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(attention_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attention_kernel<128, RT><<<grid, threads, smem, stream>>>(p);
+        attention_kernel<128><<<grid, threads, smem, stream>>>(p);
     }
     return cudaGetLastError();
 }
