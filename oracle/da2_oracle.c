@@ -549,6 +549,40 @@ int oracle_assign(int BH, int R, const double* A, int bp8, int bp4, uint8_t* pre
 }
 
 /* ------------------------------------------------------------------------ */
+/* 4b. Per-query-row ranking option (a reading of "ranks blocks per query    */
+/* row"; the pages rank all R^2 pairs of a head, item 4): the R key blocks  */
+/* of each query block a are sorted by A descending, ties to the smaller     */
+/* key block b.  Quotas per row: T8 = floor(R bp8/10^4), Tkeep =             */
+/* floor(R (bp8+bp4)/10^4); rank < T8 -> 8, rank < Tkeep -> 4, else skip.    */
+/* Outputs as oracle_assign.                                                 */
+/* ------------------------------------------------------------------------ */
+int oracle_assign_rows(int BH, int R, const double* A, int bp8, int bp4, uint8_t* prec, int* cnt,
+                       uint16_t* kidx) {
+    if (bp8 < 0 || bp4 < 0 || bp8 + bp4 > 10000) return -1;
+    long long T8 = (long long)R * bp8 / 10000, Tk = (long long)R * (bp8 + bp4) / 10000;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < BH; ++bh) {
+        o_pair* pr = (o_pair*)malloc(sizeof(o_pair) * R);
+        for (int a = 0; a < R; ++a) {
+            size_t row = (size_t)bh * R + a;
+            const double* Ar = A + row * R;
+            for (int b = 0; b < R; ++b) { pr[b].a = Ar[b]; pr[b].idx = b; }
+            qsort(pr, (size_t)R, sizeof(o_pair), pair_cmp);
+            uint8_t* P = prec + row * R;
+            for (int r = 0; r < R; ++r) P[pr[r].idx] = (r < T8) ? 8 : (r < Tk ? 4 : 0);
+            int n8 = 0, n4 = 0;
+            uint16_t* L = kidx + row * R;
+            for (int b = 0; b < R; ++b) if (P[b] == 8) L[n8++] = (uint16_t)b;
+            for (int b = 0; b < R; ++b) if (P[b] == 4) L[n8 + n4++] = (uint16_t)b;
+            cnt[row] = n8;
+            cnt[(size_t)BH * R + row] = n4;
+        }
+        free(pr);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* 6. Block-sparse attention with shared normalization (App. B.3, C.1;       */
 /*    Sec. 3.3 phased execution and cross-precision accumulation).           */
 /* For each valid query u of block a, in fp64:                               */

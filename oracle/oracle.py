@@ -56,6 +56,7 @@ def lib():
         L.oracle_prepare.argtypes = [i] * 6 + [P] * 3 + [P] * 13
         L.oracle_draft.argtypes = [i, i, i, P, ctypes.c_double, P]
         L.oracle_assign.argtypes = [i, i, P, i, i, P, P, P]
+        L.oracle_assign_rows.argtypes = [i, i, P, i, i, P, P, P]
         L.oracle_attention.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P, P]
         L.oracle_dense.argtypes = [i, i, i, P, P, P, P]
         L.oracle_num_threads.restype = i
@@ -185,12 +186,15 @@ class Plan:
     kidx: np.ndarray   # u16 [B,H,R,R] row a: 8-bit blocks asc, then 4-bit blocks asc
 
 
-def assign(A: np.ndarray, bp8: int, bp4: int) -> Plan:
+def assign(A: np.ndarray, bp8: int, bp4: int, per_row: bool = False) -> Plan:
+    """Precision of every pair: ranking of all R^2 pairs of a head (the pages),
+    or with per_row of the R key blocks of each query block."""
     A = np.ascontiguousarray(A, np.float64)
     B, H, R, _ = A.shape
     plan = Plan(prec=np.zeros((B, H, R, R), np.uint8), cnt=np.zeros((2, B, H, R), np.int32),
                 kidx=np.zeros((B, H, R, R), np.uint16))
-    if lib().oracle_assign(B * H, R, _p(A), int(bp8), int(bp4), _p(plan.prec), _p(plan.cnt), _p(plan.kidx)):
+    fn = lib().oracle_assign_rows if per_row else lib().oracle_assign
+    if fn(B * H, R, _p(A), int(bp8), int(bp4), _p(plan.prec), _p(plan.cnt), _p(plan.kidx)):
         raise ValueError("bad budget")
     return plan
 
@@ -222,10 +226,10 @@ def dense(q, k, v) -> np.ndarray:
     return out
 
 
-def run(q, k, v, F, Hv, Wv, bp8, bp4, lam=0.2, flags=7):
+def run(q, k, v, F, Hv, Wv, bp8, bp4, lam=0.2, flags=7, per_row=False):
     """Whole pipeline: prepare -> draft -> assign -> attention."""
     prep = prepare(q, k, v, F, Hv, Wv)
     A = draft(prep.desc, lam)
-    plan = assign(A, bp8, bp4)
+    plan = assign(A, bp8, bp4, per_row)
     out = attention(q, k, v, F, Hv, Wv, prep, plan, flags)
     return prep, A, plan, out

@@ -229,3 +229,58 @@ def test_quantization_error_bounds():
         # plus the group scale's own rounding (relative 2^-4) at saturation
         bound = np.repeat(sf, 16, axis=1) * g * 1.0 + np.abs(x) * 2.0 ** -4 + 1e-12
         assert np.all(np.abs(x4 - x) <= bound)
+
+
+def _brute_assign_rows(A, bp8, bp4):
+    R = A.shape[0]
+    T8, Tk = R * bp8 // 10000, R * (bp8 + bp4) // 10000
+    prec = np.zeros((R, R), np.uint8)
+    for a in range(R):
+        order = sorted(range(R), key=lambda b: (-A[a, b], b))
+        for r, b in enumerate(order):
+            prec[a, b] = 8 if r < T8 else (4 if r < Tk else 0)
+    return prec
+
+
+@pytest.mark.parametrize("bp8,bp4", [(2500, 2500), (0, 0), (10000, 0), (0, 10000), (1000, 3000), (700, 600)])
+def test_assign_rows_matches_brute_force_sort(bp8, bp4):
+    q, k, v, (F, Hv, Wv) = _tiny(3, 1, 2, 64, 6, 16, 16)
+    prep = O.prepare(q, k, v, F, Hv, Wv)
+    A = O.draft(prep.desc, 0.2)
+    plan = O.assign(A, bp8, bp4, per_row=True)
+    R = A.shape[-1]
+    for h in range(2):
+        ref = _brute_assign_rows(A[0, h], bp8, bp4)
+        assert np.array_equal(plan.prec[0, h], ref)
+        for a in range(R):
+            # per-row quotas, exact
+            assert (ref[a] == 8).sum() == R * bp8 // 10000
+            assert (ref[a] == 4).sum() == R * (bp8 + bp4) // 10000 - R * bp8 // 10000
+            n8, n4 = plan.cnt[0, 0, h, a], plan.cnt[1, 0, h, a]
+            row = plan.kidx[0, h, a]
+            assert list(row[:n8]) == list(np.nonzero(ref[a] == 8)[0])
+            assert list(row[n8:n8 + n4]) == list(np.nonzero(ref[a] == 4)[0])
+            # precision by mass inside each row
+            Ar = A[0, h, a]
+            if (ref[a] == 8).any() and (ref[a] == 4).any():
+                assert Ar[ref[a] == 8].min() >= Ar[ref[a] == 4].max()
+            if (ref[a] == 4).any() and (ref[a] == 0).any():
+                assert Ar[ref[a] == 4].min() >= Ar[ref[a] == 0].max()
+
+
+def test_assign_rows_ties_resolved_by_key_block():
+    F, Hv, Wv = 4, 16, 16
+    q, k, v = make_qkv(1, 1, F * Hv * Wv, 64, 4)
+    regs = _regions(F, Hv, Wv)
+    for t in (q, k):
+        base = t[0, 0, regs[0]].clone()
+        for toks in regs:
+            t[0, 0, toks] = base
+    prep = O.prepare(q, k, v, F, Hv, Wv)
+    A = O.draft(prep.desc, 0.2)
+    plan = O.assign(A, 2500, 2500, per_row=True)
+    R = A.shape[-1]
+    T8, Tk = R * 2500 // 10000, R * 5000 // 10000
+    for a in range(R):
+        row = plan.prec[0, 0, a]
+        assert np.all(row[:T8] == 8) and np.all(row[T8:Tk] == 4) and np.all(row[Tk:] == 0)
