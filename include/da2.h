@@ -66,6 +66,10 @@ typedef struct {
     int bp_fp8;    /* basis points of the R^2 region pairs of each head kept in FP8 */
     int bp_fp4;    /* basis points kept in NVFP4; bp_fp8 + bp_fp4 <= 10000; the rest is skipped */
     double lambda; /* max-pool branch weight of the draft map (Eq. 3); 0 = average only */
+    int per_row;   /* 0: rank all R^2 pairs of a head (DraftAttention2, Sec. 3.1 and App. C.1
+                      "ranks all video-region pairs within each head").  1: rank the R key
+                      blocks of each query block separately, quotas floor(R bp/10^4) per row
+                      (a reading of a per-query-row ranking; ties to the smaller key block). */
 } da2_budget;
 
 typedef struct da2_ctx* da2_handle;

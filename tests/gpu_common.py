@@ -36,11 +36,11 @@ def inputs(B, H, d, F, Hv, Wv, seed=0):
     return make_qkv(B, H, F * Hv * Wv, d, seed)
 
 
-def gpu_run(B, H, d, F, Hv, Wv, bp8, bp4, lam=0.2, seed=0, qkv=None):
+def gpu_run(B, H, d, F, Hv, Wv, bp8, bp4, lam=0.2, seed=0, qkv=None, per_row=False):
     q, k, v = qkv if qkv is not None else inputs(B, H, d, F, Hv, Wv, seed)
     m = da2.DA2(B, H, d, F, Hv, Wv)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    out, prep, plan = m.forward(qd, kd, vd, bp8, bp4, lam)
+    out, prep, plan = m.forward(qd, kd, vd, bp8, bp4, lam, per_row=per_row)
     torch.cuda.synchronize()
     m.check_status()
     res = {

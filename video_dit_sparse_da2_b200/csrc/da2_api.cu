@@ -213,6 +213,7 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
     a.bp8 = budget->bp_fp8;
     a.bp4 = budget->bp_fp4;
     a.lambda = budget->lambda;
+    a.per_row = budget->per_row;
     a.desc = prep->desc;
     a.A = plan->A;
     a.prec = plan->prec;

@@ -39,6 +39,7 @@ struct PlanArgs {
     int BH, R, d;
     int bp8, bp4;
     double lambda;
+    int per_row;             // 1: quotas and ranking per query block instead of per head
     const double* desc;      // [4][BH][R][d]
     double* A;               // [BH][R][R] (first holds the average-branch logits)
     double* Lmax;            // [BH][R][R] max-branch logits (scratch)

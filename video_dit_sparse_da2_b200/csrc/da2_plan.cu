@@ -473,6 +473,80 @@ __global__ void __launch_bounds__(128) classify_kernel(PlanArgs p) {
     }
 }
 
+// ---------------------------------------------------------------- per-row ranking
+// Ranking option per query block (a reading of a per-query-row ranking; the
+// pages rank all R^2 pairs of a head): one CTA per row sorts the row's R keys
+// (A bits descending, then key block ascending; A >= 0, so its bits order as
+// the values) with a bitonic network in shared memory, gives rank r the
+// precision 8 (r < T8), 4 (r < Tkeep) or 0, and writes the row's lists as the
+// classification does.  Padding keys (bits 0, index 0xFFFF) sort last.
+constexpr int kRowRankThreads = 256;
+
+__global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, int P, long long T8, long long Tk) {
+    extern __shared__ __align__(16) unsigned char rr_smem[];
+    unsigned long long* key = reinterpret_cast<unsigned long long*>(rr_smem);  // [P]
+    uint16_t* idx = reinterpret_cast<uint16_t*>(key + P);                      // [P]
+    uint8_t* prec_s = reinterpret_cast<uint8_t*>(idx + P);                     // [P]
+    const int R = p.R, tid = threadIdx.x;
+    const size_t row = blockIdx.x;
+    const double* Arow = p.A + row * R;
+    for (int i = tid; i < P; i += kRowRankThreads) {
+        key[i] = i < R ? (unsigned long long)__double_as_longlong(Arow[i]) : 0ull;
+        idx[i] = i < R ? (uint16_t)i : (uint16_t)0xFFFF;
+    }
+    __syncthreads();
+    // x before y in the ranking
+    auto before = [&](int x, int y) { return key[x] > key[y] || (key[x] == key[y] && idx[x] < idx[y]); };
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += kRowRankThreads) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool up = (i & k) == 0;  // this block puts the ranking order first
+                    if (up ? before(l, i) : before(i, l)) {
+                        const unsigned long long tk = key[i];
+                        key[i] = key[l];
+                        key[l] = tk;
+                        const uint16_t ti = idx[i];
+                        idx[i] = idx[l];
+                        idx[l] = ti;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int r = tid; r < R; r += kRowRankThreads) prec_s[idx[r]] = r < T8 ? 8 : (r < Tk ? 4 : 0);
+    __syncthreads();
+    uint8_t* prow = p.prec + row * R;
+    for (int b = tid; b < R; b += kRowRankThreads) prow[b] = prec_s[b];
+    if (tid < 32) {
+        const int lane = tid;
+        const unsigned lt = (1u << lane) - 1u;
+        uint16_t* krow = p.kidx + row * R;
+        int n8 = 0;
+        for (int b0 = 0; b0 < R; b0 += 32) {
+            const int b = b0 + lane;
+            const bool is8 = b < R && prec_s[b] == 8;
+            const unsigned m = __ballot_sync(0xffffffffu, is8);
+            if (is8) krow[n8 + __popc(m & lt)] = (uint16_t)b;
+            n8 += __popc(m);
+        }
+        int n4 = 0;
+        for (int b0 = 0; b0 < R; b0 += 32) {
+            const int b = b0 + lane;
+            const bool is4 = b < R && prec_s[b] == 4;
+            const unsigned m = __ballot_sync(0xffffffffu, is4);
+            if (is4) krow[n8 + n4 + __popc(m & lt)] = (uint16_t)b;
+            n4 += __popc(m);
+        }
+        if (lane == 0) {
+            p.cnt[row] = n8;
+            p.cnt[(size_t)p.BH * R + row] = n4;
+        }
+    }
+}
+
 constexpr int kSelectPasses = 8;  // 12-bit digits cover the 96-bit key
 
 }  // namespace
@@ -535,6 +609,18 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     }
     softmax_kernel<<<(unsigned)((size_t)BH * R), kSoftThreads, smem, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.per_row) {
+        // ranking per query block: quotas per row, no selection passes
+        int P = 1;
+        while (P < R) P <<= 1;
+        const size_t rsm = (size_t)P * (sizeof(unsigned long long) + sizeof(uint16_t) + 1);
+        const long long T8r = (long long)R * p.bp8 / 10000, Tkr = (long long)R * (p.bp8 + p.bp4) / 10000;
+        if ((e = cudaFuncSetAttribute(row_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm)) !=
+            cudaSuccess)
+            return e;
+        row_rank_kernel<<<(unsigned)((size_t)BH * R), kRowRankThreads, rsm, stream>>>(p, P, T8r, Tkr);
+        return cudaGetLastError();
+    }
     select_init_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(p, T8, Tk);
     // about two 1024-thread CTAs per multiprocessor over all heads, so that
     // each CTA flushes its shared histogram once for many keys

@@ -29,7 +29,8 @@ class Shape(ctypes.Structure):
 
 
 class Budget(ctypes.Structure):
-    _fields_ = [("bp_fp8", ctypes.c_int), ("bp_fp4", ctypes.c_int), ("lam", ctypes.c_double)]
+    _fields_ = [("bp_fp8", ctypes.c_int), ("bp_fp4", ctypes.c_int), ("lam", ctypes.c_double),
+                ("per_row", ctypes.c_int)]
 
 
 _SIZE_FIELDS = ("desc", "q8", "k8", "v8", "q4", "k4", "v4", "sfq", "sfk", "sfv", "scale", "vmax",
@@ -180,12 +181,14 @@ class DA2:
         _check(lib().da2_prepare(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), _strides(q),
                                  ctypes.byref(prep.ptrs()), _stream_ptr(stream)), "da2_prepare")
 
-    def plan(self, prep: Prepared, plan: Plan, bp8: int, bp4: int, lam: float = 0.2, stream=None):
-        b = Budget(int(bp8), int(bp4), float(lam))
+    def plan(self, prep: Prepared, plan: Plan, bp8: int, bp4: int, lam: float = 0.2, stream=None,
+             per_row: bool = False):
+        b = Budget(int(bp8), int(bp4), float(lam), int(bool(per_row)))
         _check(lib().da2_plan(self.handle, ctypes.byref(prep.ptrs()), ctypes.byref(b), ctypes.byref(plan.ptrs()),
                               _stream_ptr(stream)), "da2_plan")
 
-    def plan_static(self, prep: Prepared, plan: Plan, bp8: int, bp4: int, lam: float = 0.2, stream=None):
+    def plan_static(self, prep: Prepared, plan: Plan, bp8: int, bp4: int, lam: float = 0.2, stream=None,
+                    per_row: bool = False):
         """Routing without a caller scratch buffer (da2_plan_static): for callers
         that cannot allocate device memory, e.g. while capturing a CUDA graph.
         Writes plan.bufs' prec / cnt / kidx / A; plan.bufs["scratch"] is unused."""
@@ -194,7 +197,7 @@ class DA2:
         if need > limit:
             raise DA2Error(f"da2_plan_static: this shape needs {need} bytes of working memory, "
                            f"more than the library's fixed {limit} bytes; use plan() with a scratch buffer")
-        b = Budget(int(bp8), int(bp4), float(lam))
+        b = Budget(int(bp8), int(bp4), float(lam), int(bool(per_row)))
         bufs = plan.bufs
         _check(lib().da2_plan_static(self.handle, ctypes.byref(prep.ptrs()), ctypes.byref(b), bufs["prec"].data_ptr(),
                                      bufs["cnt"].data_ptr(), bufs["kidx"].data_ptr(), bufs["A"].data_ptr(),
@@ -208,12 +211,12 @@ class DA2:
     def check_status(self, stream=None):
         _check(lib().da2_check_device_status(self.handle, _stream_ptr(stream)), "device status")
 
-    def forward(self, q, k, v, bp8, bp4, lam=0.2, out=None, prep=None, plan=None, stream=None):
+    def forward(self, q, k, v, bp8, bp4, lam=0.2, out=None, prep=None, plan=None, stream=None, per_row=False):
         """prepare -> plan -> attention; returns (out, prep, plan)."""
         prep = prep or self.alloc_prepared(q.device)
         plan = plan or self.alloc_plan(q.device)
         out = torch.empty_like(q) if out is None else out
         self.prepare(q, k, v, prep, stream)
-        self.plan(prep, plan, bp8, bp4, lam, stream)
+        self.plan(prep, plan, bp8, bp4, lam, stream, per_row)
         self.attention(prep, plan, out, stream)
         return out, prep, plan
