@@ -175,3 +175,58 @@ def test_zero_values_give_zero_output():
     v = torch.zeros_like(v)
     _, _, _, out = O.run(q, k, v, F, HV, WV, 2500, 2500)
     assert not out.any()
+
+
+@pytest.mark.parametrize("bp8,bp4", [(10000, 0), (0, 10000), (2500, 2500), (1000, 3000)])
+def test_quantized_weights_closed_form_uniform_scores(bp8, bp4):
+    # K = 0: every score of a row ties, so p = 1 for every valid key.  One
+    # entry of +8 in every V tile gives every tile the head's maximum amax,
+    # so every tile scale equals the head maximum: s8_V = vmax8 and g4_V =
+    # vmax4, hence ratio8 = s8/sigma8 ~ 448 and ratio4 = g4/sigma4 ~ 2688
+    # with sigma8 = vmax8/448, sigma4 = vmax4/2688 (reading 9).  The weights
+    # of p = 1 then follow from the formats alone: FP8 e4m3(ratio8) = 448
+    # (the largest e4m3 value); NVFP4: the group scale e4m3(ratio4/6) = 448
+    # and e2m1(ratio4 * (1/448)) = 6, so the weight is 6 * 448 = 2688.  Each
+    # output is (f8 * sum of the FP8-kept dequantized values + f4 * sum of the
+    # NVFP4-kept ones) / (number of kept valid keys), f8 = 448 sigma8 / s8 and
+    # f4 = 2688 sigma4 / g4 (both 1 up to one fp32 rounding), across the
+    # phase switch and its change of units.
+    f32 = np.float32
+    q, k, v = _qkv(6)
+    k = torch.zeros_like(k)
+    st, na = O.slot_tokens(F, HV, WV)
+    R, d = len(na), q.shape[-1]
+    for a in range(R):
+        v[:, :, st[a * 64], 0] = 8.0
+    assert float(v.float().abs().max()) == 8.0
+    prep, A, plan, out = O.run(q, k, v, F, HV, WV, bp8, bp4, flags=7)
+    e4, e2 = _dequant_tables()
+    for h in range(2):
+        s8 = f32(prep.s8[2, 0, h, 0])
+        g4 = f32(prep.g4[2, 0, h, 0])
+        assert np.all(prep.s8[2, 0, h] == s8) and np.all(prep.g4[2, 0, h] == g4)
+        sig8, sig4 = f32(prep.vmax[0, 0, h]) / f32(448), f32(prep.vmax[1, 0, h]) / f32(2688)
+        r8, r4 = f32(s8 / sig8), f32(g4 / sig4)
+        assert O.e4m3_decode(O.e4m3_encode(float(r8))) == 448.0
+        assert O.e4m3_decode(O.e4m3_encode(float(f32(r4 / f32(6))))) == 448.0
+        assert O.e2m1_decode(O.e2m1_encode(float(f32(r4 * f32(1.0 / 448.0))))) == 6.0
+        f8 = 448.0 * float(sig8) / float(s8)
+        f4 = 2688.0 * float(sig4) / float(g4)
+        dq = {}
+        for b in range(R):
+            dq[8, b] = (e4[prep.v8t[0, h, b]] * float(s8)).T[:na[b]]
+            sv = np.repeat(e4[prep.sfv[0, h, b]], 16, 1)
+            dq[4, b] = ((e2[prep.v4t[0, h, b]] * sv) * float(g4)).T[:na[b]]
+        for a in range(R):
+            toks = st[a * 64:a * 64 + na[a]]
+            num, cnt = np.zeros(d), 0
+            for b in range(R):
+                p = plan.prec[0, h, a, b]
+                if p == 8:
+                    num += f8 * dq[8, b].sum(0)
+                elif p == 4:
+                    num += f4 * dq[4, b].sum(0)
+                if p:
+                    cnt += na[b]
+            ref = num / cnt if cnt else np.zeros(d)
+            np.testing.assert_allclose(out[0, h, toks], np.broadcast_to(ref, (len(toks), d)), rtol=1e-12, atol=1e-12)
