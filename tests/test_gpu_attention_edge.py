@@ -69,3 +69,19 @@ def test_attention_zero_keys_uniform_weights():
     k = torch.zeros_like(k)
     res = gpu_run(B, H, d, F, Hv, Wv, 2500, 2500, qkv=(q, k, v))
     _check(res, q, k, v, F, Hv, Wv, 2500, 2500)
+
+
+@pytest.mark.parametrize("bp", [(10000, 0), (0, 10000), (2500, 2500)])
+def test_attention_saturated_weights(bp):
+    # zero keys (every p = 1) and every V tile at the head maximum: the FP8
+    # weights sit at the largest e4m3 value and the NVFP4 group scales at the
+    # largest ue4m3 value, with e2m1 codes 6
+    B, H, d, F, Hv, Wv = SHAPES["tiny"]
+    q, k, v = inputs(B, H, d, F, Hv, Wv)
+    k = torch.zeros_like(k)
+    v = v.clone()
+    st, na = O.slot_tokens(F, Hv, Wv)
+    for a in range(len(na)):
+        v[:, :, st[a * 64], 0] = 8.0
+    res = gpu_run(B, H, d, F, Hv, Wv, *bp, qkv=(q, k, v))
+    _check(res, q, k, v, F, Hv, Wv, *bp)
