@@ -475,53 +475,97 @@ __global__ void __launch_bounds__(128) classify_kernel(PlanArgs p) {
 
 // ---------------------------------------------------------------- per-row ranking
 // Ranking option per query block (a reading of a per-query-row ranking; the
-// pages rank all R^2 pairs of a head): one CTA per row sorts the row's R keys
-// (A bits descending, then key block ascending; A >= 0, so its bits order as
-// the values) with a bitonic network in shared memory, gives rank r the
-// precision 8 (r < T8), 4 (r < Tkeep) or 0, and writes the row's lists as the
-// classification does.  Padding keys (bits 0, index 0xFFFF) sort last.
+// pages rank all R^2 pairs of a head).  One CTA per row finds the T8-th and
+// Tkeep-th largest 76-bit keys K = (A bits : 0xFFF - b) -- A descending, ties
+// to the smaller key block b (A >= 0, so its bits order as the values) -- by
+// a radix selection over 8-bit digits in shared memory, then gives each key
+// block 8 (K >= K_T8), 4 (K >= K_Tkeep) or 0 and writes the row's lists as the
+// classification does.
 constexpr int kRowRankThreads = 256;
+typedef unsigned __int128 u128;
 
-__global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, int P, long long T8, long long Tk) {
-    extern __shared__ __align__(16) unsigned char rr_smem[];
-    unsigned long long* key = reinterpret_cast<unsigned long long*>(rr_smem);  // [P]
-    uint16_t* idx = reinterpret_cast<uint16_t*>(key + P);                      // [P]
-    uint8_t* prec_s = reinterpret_cast<uint8_t*>(idx + P);                     // [P]
-    const int R = p.R, tid = threadIdx.x;
+__global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, long long T8, long long Tk) {
+    __shared__ unsigned hist[2][256];
+    __shared__ u128 pre[2];      // selected prefix (digits in place)
+    __shared__ int nbits[2];     // bits of the prefix already fixed
+    __shared__ long long need[2];  // rank still sought inside the prefix (1-based)
+    __shared__ uint8_t prec_s[4096];
+    const int R = p.R, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t row = blockIdx.x;
     const double* Arow = p.A + row * R;
-    for (int i = tid; i < P; i += kRowRankThreads) {
-        key[i] = i < R ? (unsigned long long)__double_as_longlong(Arow[i]) : 0ull;
-        idx[i] = i < R ? (uint16_t)i : (uint16_t)0xFFFF;
+    auto keyof = [&](int b) -> u128 {
+        return ((u128)(unsigned long long)__double_as_longlong(Arow[b]) << 12) | (u128)(0xFFFu - (unsigned)b);
+    };
+    if (tid < 2) {
+        pre[tid] = 0;
+        nbits[tid] = 0;
+        need[tid] = tid == 0 ? T8 : Tk;
     }
     __syncthreads();
-    // x before y in the ranking
-    auto before = [&](int x, int y) { return key[x] > key[y] || (key[x] == key[y] && idx[x] < idx[y]); };
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P; i += kRowRankThreads) {
-                const int l = i ^ j;
-                if (l > i) {
-                    const bool up = (i & k) == 0;  // this block puts the ranking order first
-                    if (up ? before(l, i) : before(i, l)) {
-                        const unsigned long long tk = key[i];
-                        key[i] = key[l];
-                        key[l] = tk;
-                        const uint16_t ti = idx[i];
-                        idx[i] = idx[l];
-                        idx[l] = ti;
+    for (int pass = 0; pass < 10; ++pass) {  // 76 bits in 8-bit digits (the last one 4 bits)
+        for (int i = tid; i < 2 * 256; i += kRowRankThreads) (&hist[0][0])[i] = 0u;
+        __syncthreads();
+        int w[2], pos[2];
+        bool live[2];
+        for (int t = 0; t < 2; ++t) {
+            live[t] = need[t] > 0 && nbits[t] < 76;
+            w[t] = min(8, 76 - nbits[t]);
+            pos[t] = 76 - nbits[t] - w[t];
+        }
+        if (!live[0] && !live[1]) break;  // uniform: read from shared state after the barrier
+        for (int b = tid; b < R; b += kRowRankThreads) {
+            const u128 K = keyof(b);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (!live[t]) continue;
+                const int sh = 76 - nbits[t];
+                if (sh < 128 && (K >> sh) != (pre[t] >> sh)) continue;
+                atomicAdd(&hist[t][(unsigned)(K >> pos[t]) & ((1u << w[t]) - 1u)], 1u);
+            }
+        }
+        __syncthreads();
+        if (warp < 2 && live[warp]) {
+            const int t = warp;
+            // lane covers bins [255 - 8 lane - 7, 255 - 8 lane], descending
+            const int top = 255 - 8 * lane;
+            unsigned sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += hist[t][top - i];
+            unsigned incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const unsigned excl = incl - sum;
+            const long long nd = need[t];
+            if ((long long)excl < nd && nd <= (long long)incl) {
+                long long cum = excl;
+                for (int i = 0; i < 8; ++i) {
+                    const int bin = top - i;
+                    const long long c = hist[t][bin];
+                    if (cum + c >= nd) {
+                        need[t] = nd - cum;
+                        pre[t] |= (u128)bin << pos[t];
+                        nbits[t] += w[t];
+                        break;
                     }
+                    cum += c;
                 }
             }
-            __syncthreads();
         }
+        __syncthreads();
     }
-    for (int r = tid; r < R; r += kRowRankThreads) prec_s[idx[r]] = r < T8 ? 8 : (r < Tk ? 4 : 0);
+    const u128 k8 = pre[0], kk = pre[1];
+    const bool has8 = T8 > 0, hask = Tk > 0;
+    for (int b = tid; b < R; b += kRowRankThreads) {
+        const u128 K = keyof(b);
+        prec_s[b] = (has8 && K >= k8) ? 8 : ((hask && K >= kk) ? 4 : 0);
+    }
     __syncthreads();
     uint8_t* prow = p.prec + row * R;
     for (int b = tid; b < R; b += kRowRankThreads) prow[b] = prec_s[b];
     if (tid < 32) {
-        const int lane = tid;
         const unsigned lt = (1u << lane) - 1u;
         uint16_t* krow = p.kidx + row * R;
         int n8 = 0;
@@ -611,14 +655,8 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.per_row) {
         // ranking per query block: quotas per row, no selection passes
-        int P = 1;
-        while (P < R) P <<= 1;
-        const size_t rsm = (size_t)P * (sizeof(unsigned long long) + sizeof(uint16_t) + 1);
         const long long T8r = (long long)R * p.bp8 / 10000, Tkr = (long long)R * (p.bp8 + p.bp4) / 10000;
-        if ((e = cudaFuncSetAttribute(row_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm)) !=
-            cudaSuccess)
-            return e;
-        row_rank_kernel<<<(unsigned)((size_t)BH * R), kRowRankThreads, rsm, stream>>>(p, P, T8r, Tkr);
+        row_rank_kernel<<<(unsigned)((size_t)BH * R), kRowRankThreads, 0, stream>>>(p, T8r, Tkr);
         return cudaGetLastError();
     }
     select_init_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(p, T8, Tk);
