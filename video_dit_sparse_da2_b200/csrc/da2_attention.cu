@@ -19,10 +19,13 @@
 //              Reads S from tensor memory (then releases the S buffer at
 //              once), keeps the row max m and the unquantized denominator l
 //              (App. B.3), quantizes the weights into shared memory -- FP8:
-//              e4m3 of p times the value tile scale over the phase unit;
-//              NVFP4: that product quantized per 16 keys with a ue4m3 scale --
-//              with the same fp32 rounding steps as the definition (p of the
-//              winning key is exactly 1), rescales its row of O when m grows
+//              e4m3 of p times the value tile scale over the phase unit, with
+//              the fp32 rounding steps of the definition; NVFP4: per 16 keys a
+//              ue4m3 scale from the group's largest weight (taken from the
+//              group maximum of the scores) and e2m1 codes of p * (ratio *
+//              1/scale), the definition's (p * ratio) * 1/scale reordered,
+//              equal to it whenever p is a power of two; p of the winning key
+//              is exactly 1 in both -- rescales its row of O when m grows
 //              and once at the phase switch (sigma8 -> sigma4, the change of
 //              units of Eq. 8), and in the epilogue divides by l, converts to
 //              bf16 and stores the row at its original token position.
