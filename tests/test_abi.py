@@ -61,3 +61,13 @@ def test_library_partition_matches_oracle(geom):
 def test_partition_rejects_bad_sizes():
     assert da2.lib().da2_partition(0, 4, 4, None, None) == da2.ERR_ARG
     assert da2.lib().da2_partition(1, 0, 4, None, None) == da2.ERR_ARG
+
+
+def test_budget_struct_layout_matches_header():
+    # da2_budget in include/da2.h: int bp_fp8, int bp_fp4, double lambda, int per_row
+    import ctypes
+
+    from video_dit_sparse_da2_b200 import da2
+    B = da2.Budget
+    assert [B.bp_fp8.offset, B.bp_fp4.offset, B.lam.offset, B.per_row.offset] == [0, 4, 8, 16]
+    assert ctypes.sizeof(B) == 24
