@@ -166,8 +166,10 @@ int da2_prepare(da2_handle h, const void* q, const void* k, const void* v, const
  * operation order, per-head ranking of all R^2 pairs by A (ties to the
  * smaller pair index a*R+b), quotas T8 = floor(R^2 bp_fp8/10^4),
  * Tkeep = floor(R^2 (bp_fp8+bp_fp4)/10^4); ranks below T8 -> FP8, below
- * Tkeep -> NVFP4, the rest skipped; per-row lists.  Errors: DA2_ERR_ARG for
- * a budget outside [0, 10000] or lambda outside [0, 1]. */
+ * Tkeep -> NVFP4, the rest skipped; per-row lists.  With budget->per_row = 1
+ * the ranking and the quotas floor(R bp/10^4) are per query block instead.
+ * Errors: DA2_ERR_ARG for a budget outside [0, 10000], lambda outside [0, 1]
+ * or per_row other than 0 / 1. */
 int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, const da2_plan_bufs* plan,
              void* stream);
 

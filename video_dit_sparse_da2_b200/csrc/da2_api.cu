@@ -206,6 +206,7 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
     if (!h || !prepared_ok(prep) || !budget || !plan_ok(plan)) return DA2_ERR_ARG;
     if (budget->bp_fp8 < 0 || budget->bp_fp4 < 0 || budget->bp_fp8 + budget->bp_fp4 > 10000) return DA2_ERR_ARG;
     if (!(budget->lambda >= 0.0 && budget->lambda <= 1.0)) return DA2_ERR_ARG;
+    if (budget->per_row != 0 && budget->per_row != 1) return DA2_ERR_ARG;
     da2::PlanArgs a{};
     a.BH = h->shape.B * h->shape.H;
     a.R = h->R;
