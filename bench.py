@@ -31,7 +31,7 @@ METRIC = "ms/call and dense-equiv TFLOPS at 1 B200; % of mixed FP8/FP4 tensor ro
 # DRAM bytes (read + write) of one attention launch, from the ncu capture in
 # profiles/attention_kernel_wan13b_480p.md, valid for the attention sources
 # whose hash is given (the field is null for any other source or workload).
-ATTN_TRAFFIC = {"wan2.1-1.3b-480p": {"sources_sha256_16": "b34ce025aefd3c95", "bytes": 146444288 + 63652352}}
+ATTN_TRAFFIC = {"wan2.1-1.3b-480p": {"sources_sha256_16": "30c0ac47a9ec318c", "bytes": 146444288 + 63652352}}
 _ATTN_SOURCES = ("video_dit_sparse_da2_b200/csrc/da2_attention.cu", "video_dit_sparse_da2_b200/csrc/da2_common.cuh")
 
 
