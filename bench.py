@@ -28,27 +28,32 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ms/call and dense-equiv TFLOPS at 1 B200; % of mixed FP8/FP4 tensor roofline"
 
-# DRAM bytes (read + write) of one attention launch, from the ncu capture in
-# profiles/attention_kernel_wan13b_480p.md, valid for the attention sources
-# whose hash is given (the field is null for any other source or workload).
-ATTN_TRAFFIC = {"wan2.1-1.3b-480p": {"sources_sha256_16": "30c0ac47a9ec318c", "bytes": 146444288 + 63652352}}
+# DRAM bytes (read + write) of one attention launch, measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum) on the workload named, for the
+# attention sources whose hash is given; any other source or workload reports
+# null.  Filled in only from a capture of the current kernel.
+ATTN_TRAFFIC: dict = {}
 _ATTN_SOURCES = ("video_dit_sparse_da2_b200/csrc/da2_attention.cu", "video_dit_sparse_da2_b200/csrc/da2_common.cuh")
 
 
-def attention_traffic(workload: str):
+def attention_sources_hash() -> str:
     import hashlib
+    h = hashlib.sha256()
+    for f in _ATTN_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def attention_traffic(workload: str):
     rec = ATTN_TRAFFIC.get(workload)
     if rec is None:
         return None
-    h = hashlib.sha256()
-    root = os.path.dirname(os.path.abspath(__file__))
     try:
-        for f in _ATTN_SOURCES:
-            with open(os.path.join(root, f), "rb") as fh:
-                h.update(fh.read())
+        return rec["bytes"] if attention_sources_hash() == rec["sources_sha256_16"] else None
     except OSError:
         return None
-    return rec["bytes"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
+
 
 UNIT = "TFLOPS (dense-equivalent, whole job)"
 
@@ -73,6 +78,9 @@ class Clocks:
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
 
+    PERIOD_MS = 20
+    MIN_SAMPLES = 5
+
     def __init__(self, index: int):
         self.index = index
         self.proc = None
@@ -83,7 +91,7 @@ class Clocks:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -110,7 +118,11 @@ class Clocks:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
         loaded = [s for s in sm if s > 0.5 * mx] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+        rec = {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+               "period_ms": self.PERIOD_MS}
+        if len(rows) < self.MIN_SAMPLES:
+            rec["insufficient"] = f"{len(rows)} samples (< {self.MIN_SAMPLES}) during the timed region"
+        return rec
 
 
 def kept_pair_counts(plan_cnt, B, H, R):
@@ -176,6 +188,7 @@ def run_ours(args, w, rank, world):
     barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
+    time.sleep(0.3)  # nvidia-smi is sampling before the timed region opens
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -252,58 +265,62 @@ def run_ours(args, w, rank, world):
                 h2d=3 * q.numel() * 2, d2h=out.numel() * 2)
 
 
-def oracle_sample(w, budget_s: float = 20.0):
-    """Time the oracle on a bounded sample of one call of workload w.
+class OracleSampler:
+    """Times the oracle on bounded samples of one call of workload w.
 
-    Sample: prepare + draft + assign for `hs` heads (all heads when cheap),
-    attention for a fixed set of query blocks of those heads; the per-call
-    time is extrapolated linearly to all heads and blocks."""
-    import numpy as np
+    The inputs (the same seeded tensors as the device run, restricted to the
+    first `hs` heads, hs = min(H, host threads)) are drawn once.  A sample
+    runs prepare + draft + assign on those heads and attention on a doubling
+    number of random query blocks per head until its time budget is used;
+    the per-call time is extrapolated linearly to all heads and blocks."""
 
-    from oracle import oracle as O
-    from video_dit_sparse_da2_b200.inputs import make_qkv
+    def __init__(self, w):
+        from oracle import oracle as O
+        from video_dit_sparse_da2_b200.inputs import make_qkv
+        self.O, self.w = O, w
+        self.cores = O.num_threads()
+        self.hs = max(1, min(w.H, self.cores))
+        self.qkv = make_qkv(w.B, self.hs, w.N, w.d, seed=0)
+        self.rng = __import__("numpy").random.default_rng(0)
 
-    cores = O.num_threads()
-    hs = max(1, min(w.H, cores))
-    q, k, v = make_qkv(w.B, hs, w.N, w.d, seed=0)
-    t0 = time.perf_counter()
-    prep = O.prepare(q, k, v, w.F, w.Hv, w.Wv)
-    A = O.draft(prep.desc, w.lam)
-    plan = O.assign(A, w.bp8, w.bp4)
-    t_pp = time.perf_counter() - t0
-    R = A.shape[-1]
-    nblk = 1
-    total_blocks = 0
-    t_att = 0.0
-    sel_all = np.zeros((w.B, hs, R), np.uint8)
-    rng = np.random.default_rng(0)
-    while True:
-        sel = np.zeros((w.B, hs, R), np.uint8)
-        for h in range(hs):
-            sel[0, h, rng.choice(R, size=min(nblk, R), replace=False)] = 1
-        t1 = time.perf_counter()
-        O.attention(q, k, v, w.F, w.Hv, w.Wv, prep, plan, blocks=sel)
-        dt = time.perf_counter() - t1
-        t_att += dt
-        total_blocks += int(sel.sum())
-        sel_all |= sel
-        if t_pp + t_att > budget_s or nblk >= R or dt * 4 > budget_s:
-            break
-        nblk *= 2
-    per_block = t_att / total_blocks * hs  # seconds per block with hs blocks running in parallel threads
-    t_call = (t_pp * w.H / hs) + per_block * R * w.H / hs
-    sample = (f"oracle (C, fp64, OpenMP {cores} threads): prepare+draft+assign on {hs} of {w.H} heads "
-              f"({t_pp:.1f} s), attention on {total_blocks} of {w.H * R} query blocks ({t_att:.1f} s); "
-              f"per-call time extrapolated linearly to all heads and blocks: {t_call:.1f} s")
-    return t_call, cores, sample
+    def sample(self, budget_s: float):
+        import numpy as np
+        O, w, hs = self.O, self.w, self.hs
+        q, k, v = self.qkv
+        t0 = time.perf_counter()
+        prep = O.prepare(q, k, v, w.F, w.Hv, w.Wv)
+        A = O.draft(prep.desc, w.lam)
+        plan = O.assign(A, w.bp8, w.bp4)
+        t_pp = time.perf_counter() - t0
+        R = A.shape[-1]
+        nblk, total_blocks, t_att = 1, 0, 0.0
+        while True:
+            sel = np.zeros((w.B, hs, R), np.uint8)
+            for h in range(hs):
+                sel[0, h, self.rng.choice(R, size=min(nblk, R), replace=False)] = 1
+            t1 = time.perf_counter()
+            O.attention(q, k, v, w.F, w.Hv, w.Wv, prep, plan, blocks=sel)
+            dt = time.perf_counter() - t1
+            t_att += dt
+            total_blocks += int(sel.sum())
+            if t_pp + t_att > budget_s or nblk >= R or dt * 4 > budget_s:
+                break
+            nblk *= 2
+        per_block = t_att / total_blocks * hs  # seconds per block with hs blocks running in parallel threads
+        t_call = (t_pp * w.H / hs) + per_block * R * w.H / hs
+        desc = (f"oracle (C, fp64, OpenMP {self.cores} threads): prepare+draft+assign on {hs} of {w.H} heads "
+                f"({t_pp:.1f} s), attention on {total_blocks} of {w.H * R} query blocks ({t_att:.1f} s); "
+                f"per-call time extrapolated linearly to all heads and blocks: {t_call:.1f} s")
+        return t_call, desc
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=250)  # about 1 s timed on the default workload
+    ap.add_argument("--steps", type=int, default=20)  # about 1.2 s timed on the default workload
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="wan2.1-1.3b-480p")
+    # the largest workload that fits one GPU (N = 118,800 tokens, 24 heads)
+    ap.add_argument("--workload", default="hunyuanvideo-720p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -324,14 +341,16 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        # one short untimed sample loads the oracle, then K timed samples of
-        # about 60 s of CPU work in total; the line reports their median
-        oracle_sample(w, budget_s=1.0)
-        per = max(3.0, 60.0 / max(1, args.steps))
-        runs = [oracle_sample(w, budget_s=per) for _ in range(args.steps)]
+        # inputs drawn once; one short untimed sample loads the oracle, then K
+        # timed samples of about 60 s of CPU work in total; the line reports
+        # their median
+        sampler = OracleSampler(w)
+        sampler.sample(budget_s=0.5)
+        per = max(2.0, 60.0 / max(1, args.steps))
+        runs = [sampler.sample(budget_s=per) for _ in range(args.steps)]
         t_call = statistics.median(r[0] for r in runs)
-        cores = runs[0][1]
-        sample = f"{args.steps} samples, median; each: " + runs[len(runs) // 2][2]
+        cores = sampler.cores
+        sample = f"{args.steps} samples, median; each: " + runs[len(runs) // 2][1]
         value = flops / t_call / 1e12
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_call * 1e3, "higher_is_better": True,
@@ -394,9 +413,10 @@ def main():
                            "peak_gbs": peaks["hbm_gbs"],
                            "frac": prep_bytes / (r["t_prep"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     if world == 1 and not args.no_cpu_baseline:
-        t_call, cores, sample = oracle_sample(w, budget_s=20.0)
-        line["cpu_baseline"] = {"value": flops / t_call / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        sampler = OracleSampler(w)
+        t_call, sample = sampler.sample(budget_s=20.0)
+        line["cpu_baseline"] = {"value": flops / t_call / 1e12, "unit": UNIT, "cores": sampler.cores,
+                                "kind": "oracle", "sample": sample}
     print(json.dumps(line), flush=True)
 
 

@@ -133,8 +133,10 @@ typedef struct {
 /* Validate the shape, build the region partition on the host (App. C.2
  * reading: balanced R_f regions, boustrophedon band walk, smallest total
  * perimeter among connected candidates) and copy the slot tables to the
- * current device.  *out receives the handle.  Errors: DA2_ERR_ARG,
- * DA2_ERR_ARCH, DA2_ERR_CUDA. */
+ * current device.  *out receives the handle.  The handle also holds a status
+ * word and a work counter that its kernels share: order the calls made on one
+ * handle (one stream, or synchronize between streams), or use one handle per
+ * stream.  Errors: DA2_ERR_ARG, DA2_ERR_ARCH, DA2_ERR_CUDA. */
 int da2_create(const da2_shape* shape, da2_handle* out);
 
 /* Host-only: the partition of a shape without a device.  Fills
@@ -195,7 +197,8 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
  *   - Every call reuses the same array and clears what must start at zero;
  *     two calls that overlap on the same GPU (different streams, threads or
  *     handles) race on it: order them.
- *   - Returns DA2_ERR_ARG, without enqueueing anything, when the shape needs
+ *   - Returns DA2_ERR_ARG, without enqueueing anything, when the current
+ *     device is not the handle's device, or when the shape needs
  *     more working memory than DA2_PLAN_STATIC_BYTES (da2_sizes' plan_scratch
  *     tells how much: about B*H*R*R*8 bytes plus 33 KB per head).  Other
  *     errors as da2_plan. */
@@ -205,13 +208,33 @@ int da2_plan_static(da2_handle h, const da2_prepared* prep, const da2_budget* bu
 /* Block-sparse mixed-precision attention (Sec. 3.3; App. B.3, C.1).  out:
  * bf16 (device), [B][H][N][d] with strides out_strides[] in elements
  * (out_strides[3] == 1); every token row is written (rows with no retained
- * valid key get zeros). */
+ * valid key get zeros).  The persistent CTAs take their work items from the
+ * handle's work counter, which the call resets on `stream`: two attention
+ * calls on one handle that overlap on different streams would share it and
+ * leave rows unwritten, so order them (or use one handle per stream). */
 int da2_attention(da2_handle h, const da2_prepared* prep, const da2_plan_bufs* plan, void* out,
                   const int64_t out_strides[4], void* stream);
 
 /* Synchronize `stream` and report whether a bounded device wait gave up
  * since the last call (DA2_ERR_TIMEOUT), clearing the flag. */
 int da2_check_device_status(da2_handle h, void* stream);
+
+/* Limit of every bounded device-side wait in the kernels launched with this
+ * handle, in nanoseconds; 0 restores the default (4 s).  A wait that reaches
+ * the limit makes its kernel stop, drain its own asynchronous copies and
+ * tensor-core work, free its tensor memory and return; the next
+ * da2_check_device_status reports DA2_ERR_TIMEOUT.  The paper has no
+ * counterpart: this is a service of the library. */
+int da2_set_wait_limit(da2_handle h, uint64_t limit_ns);
+
+/* Self-test of that failure path, with no fault and no hang: enqueues on
+ * `stream` one small kernel whose first warp waits, with limit_ns, on a
+ * device barrier that nothing arrives on, and whose second warp waits on the
+ * same barrier with a 1000 times longer limit and must stop as soon as the
+ * first gives up.  The kernel returns after about limit_ns; the next
+ * da2_check_device_status then reports DA2_ERR_TIMEOUT.  limit_ns must be in
+ * (0, 10^9], else DA2_ERR_ARG.  The paper has no counterpart. */
+int da2_selftest_wait_timeout(da2_handle h, uint64_t limit_ns, void* stream);
 
 /* Static description of a status code. */
 const char* da2_status_string(int status);

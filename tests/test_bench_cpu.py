@@ -33,9 +33,20 @@ def test_max_over_ranks_single_rank_is_identity():
     assert bench.max_over_ranks(v, 1).tolist() == [3.0, 1.0]
 
 
-def test_attention_traffic_only_for_recorded_workload():
+def test_attention_traffic_only_for_recorded_source(monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
-    assert bench.attention_traffic("cogvideox") is None
-    t = bench.attention_traffic("wan2.1-1.3b-480p")
-    assert t is None or t > 0
+    assert bench.attention_traffic("no-such-workload") is None
+    h = bench.attention_sources_hash()
+    monkeypatch.setattr(bench, "ATTN_TRAFFIC", {"w": {"sources_sha256_16": h, "bytes": 123},
+                                                "old": {"sources_sha256_16": "0" * 16, "bytes": 456}})
+    assert bench.attention_traffic("w") == 123
+    assert bench.attention_traffic("old") is None  # recorded for other attention sources
+
+
+def test_default_workload_is_largest_single_gpu_config():
+    sys.path.insert(0, ROOT)
+    from video_dit_sparse_da2_b200.inputs import ALL
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    largest = max(ALL, key=lambda w: 4 * w.B * w.H * w.N * w.N * w.d)
+    assert f'ap.add_argument("--workload", default="{largest.name}")' in src

@@ -6,7 +6,8 @@ library.  It must give exactly what da2_plan gives with a caller-provided
 scratch buffer -- the routing outputs are compared bit for bit, as every
 routing test here does -- on two calls in a row (the second call finds the
 first call's leftovers in the array), and it must refuse shapes whose working
-memory exceeds the array.
+memory exceeds the array.  Both ranking modes are covered: per head, and
+per query block (which runs a different routing kernel on the same array).
 
 This file sorts last so that a run stopping at the first failure has run
 every other test before it.
@@ -33,8 +34,9 @@ def _plan_bytes(plan, B, H, R):
     return {k: np.ascontiguousarray(v).view(np.uint8).copy() for k, v in g.items()}
 
 
+@pytest.mark.parametrize("per_row", [False, True], ids=["per-head", "per-row"])
 @pytest.mark.parametrize("case", CASES, ids=["tiny", "wan2.1-1.3b-480p"])
-def test_plan_static_matches_plan_twice(case):
+def test_plan_static_matches_plan_twice(case, per_row):
     B, H, d, F, Hv, Wv, bp8, bp4, lam = case
     m = da2.DA2(B, H, d, F, Hv, Wv)
     assert m.sizes.plan_scratch <= (32 << 20)
@@ -42,14 +44,14 @@ def test_plan_static_matches_plan_twice(case):
     prep = m.alloc_prepared()
     m.prepare(q, k, v, prep)
     ref = m.alloc_plan()
-    m.plan(prep, ref, bp8, bp4, lam)
+    m.plan(prep, ref, bp8, bp4, lam, per_row=per_row)
     torch.cuda.synchronize()
     want = _plan_bytes(ref, B, H, m.R)
     for call in range(2):
         got_plan = m.alloc_plan()
         for t in got_plan.bufs.values():
             t.fill_(0xA5)  # outputs start as garbage: everything must be written
-        m.plan_static(prep, got_plan, bp8, bp4, lam)
+        m.plan_static(prep, got_plan, bp8, bp4, lam, per_row=per_row)
         torch.cuda.synchronize()
         m.check_status()
         got = _plan_bytes(got_plan, B, H, m.R)

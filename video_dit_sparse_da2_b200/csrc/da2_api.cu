@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "../../include/da2.h"
+#include "da2_common.cuh"
 #include "da2_kernels.h"
 #include "da2_partition.h"
 
@@ -19,6 +20,7 @@ struct da2_ctx {
     int32_t* d_n_a = nullptr;              // [R]
     unsigned* d_status = nullptr;          // kernel status word
     int* d_work = nullptr;                 // attention work counter
+    unsigned long long wait_ns = DA2_WAIT_NS_DEFAULT;  // limit of the kernels' bounded waits
 };
 
 namespace {
@@ -49,6 +51,11 @@ bool plan_ok(const da2_plan_bufs* p) {
 }
 
 }  // namespace
+
+namespace da2 {
+int handle_device(const da2_ctx* h) { return h->device; }
+int record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace da2
 
 extern "C" {
 
@@ -255,7 +262,20 @@ int da2_attention(da2_handle h, const da2_prepared* prep, const da2_plan_bufs* p
     a.status = h->d_status;
     a.work_counter = h->d_work;
     a.num_sms = h->num_sms;
+    a.wait_ns = h->wait_ns;
     cudaError_t e = da2::launch_attention(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DA2_OK : cuda_fail(e);
+}
+
+int da2_set_wait_limit(da2_handle h, uint64_t limit_ns) {
+    if (!h) return DA2_ERR_ARG;
+    h->wait_ns = limit_ns ? (unsigned long long)limit_ns : DA2_WAIT_NS_DEFAULT;
+    return DA2_OK;
+}
+
+int da2_selftest_wait_timeout(da2_handle h, uint64_t limit_ns, void* stream) {
+    if (!h || limit_ns == 0 || limit_ns > 1000000000ull) return DA2_ERR_ARG;
+    cudaError_t e = da2::launch_wait_selftest(h->d_status, limit_ns, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DA2_OK : cuda_fail(e);
 }
 

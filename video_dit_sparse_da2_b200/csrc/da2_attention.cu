@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             }
             for (int j = 0; j < n_ent; ++j) {
                 const uint32_t g = gstep + j, st = g % kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status)))
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status, p.wait_ns)))
                     break;
                 const uint32_t e = warp_uniform((uint32_t)list[j]);
                 const int kb = e & 0xFFF, ph = (e >> 12) & 1;
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
         } else if (warp == kMmaWarp) {
             // ================================================== MMA issue (whole warp, one elected lane issues)
             auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-                return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, p.status));
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, p.status, p.wait_ns));
             };
             bool ok = wait_all(&bar_q, nitem & 1);
             ok = ok && wait_all(&bar_sfq, nitem & 1);
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 // S of step g and its step record.  The commit also covers every
                 // earlier MMA, in particular the PV of step g-2, the last reader
                 // of P buffer pb.
-                const bool waited = mbar_wait(&bar_s, g & 1, abort_v, p.status);
+                const bool waited = mbar_wait(&bar_s, g & 1, abort_v, p.status, p.wait_ns);
                 if (!__all_sync(0xffffffffu, waited)) {
                     ok = false;
                     break;
@@ -622,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
                 const bool need = (resc || sw) && j > 0;
                 if (__any_sync(0xffffffffu, need)) {
                     // O must hold the PV of step g-1 first
-                    const bool w2 = mbar_wait(&bar_empty[(g - 1) % kStages], ((g - 1) / kStages) & 1, abort_v, p.status);
+                    const bool w2 = mbar_wait(&bar_empty[(g - 1) % kStages], ((g - 1) / kStages) & 1, abort_v, p.status, p.wait_ns);
                     if (!__all_sync(0xffffffffu, w2)) ok = false;
                     if (ok) {
                         tc_fence_after();
@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
             const bool have = n_ent > 0 && ok;
             if (have) {
                 const uint32_t g = gstep + n_ent - 1;
-                if (!mbar_wait(&bar_empty[g % kStages], (g / kStages) & 1, abort_v, p.status)) ok = false;
+                if (!mbar_wait(&bar_empty[g % kStages], (g / kStages) & 1, abort_v, p.status, p.wait_ns)) ok = false;
                 tc_fence_after();
                 const float unit = n_ent > n8e ? sig4 : sig8;
                 o_scale = lt > 0.0f ? __fdiv_rn(unit, lt) : 0.0f;
@@ -703,13 +703,13 @@ __global__ void __launch_bounds__(kThreads, 2) attention_kernel(AttnArgs p) {
     __syncthreads();
     if (warp == kMmaWarp && mma_issued) {
         tc_commit_w(&bar_drain);
-        if (lane == 0 && !mbar_wait_drain(&bar_drain, 0)) atomicOr(p.status, DA2_DEV_TIMEOUT);
+        if (lane == 0 && !mbar_wait_drain(&bar_drain, 0, p.wait_ns)) atomicOr(p.status, DA2_DEV_TIMEOUT);
     }
     if (warp == kLoadWarp && lane == 0) {
         // every issued stage fill must have landed before the CTA exits
         for (uint32_t k = 0; k < loads_issued && k < (uint32_t)kStages; ++k) {
             const uint32_t g = loads_issued - 1 - k, st = g % kStages;
-            if (!mbar_wait_drain(&bar_full[st], (g / kStages) & 1)) atomicOr(p.status, DA2_DEV_TIMEOUT);
+            if (!mbar_wait_drain(&bar_full[st], (g / kStages) & 1, p.wait_ns)) atomicOr(p.status, DA2_DEV_TIMEOUT);
         }
     }
     tc_fence_before();

@@ -13,9 +13,9 @@
 #define DA2_DEV_TIMEOUT 1u
 #define DA2_DEV_BADINDEX 2u
 
-// A device-side wait is declared stuck after this many nanoseconds (far
-// beyond any legitimate wait in these kernels).
-#define DA2_WAIT_NS 4000000000ull
+// Default limit of a device-side wait, in nanoseconds (far beyond any
+// legitimate wait in these kernels); a handle can set another one.
+#define DA2_WAIT_NS_DEFAULT 4000000000ull
 // Suspend-time hint of one mbarrier try_wait: the waiting thread sleeps in
 // hardware until the phase completes or this many nanoseconds pass.
 #define DA2_SUSPEND_NS 100000u
@@ -66,27 +66,27 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 // Bounded wait: returns false (and sets *status) when the barrier does not
-// complete the given phase within DA2_WAIT_NS, or when another warp already
+// complete the given phase within limit_ns, or when another warp already
 // gave up (*abort set).  The thread sleeps inside try_wait between checks.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned* status) {
+                                          unsigned* status, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait_sleep(bar, parity, DA2_SUSPEND_NS)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > DA2_WAIT_NS) break;
+        if (globaltimer_ns() - t0 > limit_ns) break;
     }
     *abort = 1;
     atomicOr(status, DA2_DEV_TIMEOUT);
     return false;
 }
 // Bounded wait without the abort short-cut (used to drain own async work).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait_sleep(bar, parity, DA2_SUSPEND_NS)) return true;
-        if (globaltimer_ns() - t0 > DA2_WAIT_NS) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 

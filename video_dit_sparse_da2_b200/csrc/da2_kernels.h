@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+struct da2_ctx;
+
 namespace da2 {
 
 struct PrepareArgs {
@@ -71,7 +73,16 @@ struct AttnArgs {
     unsigned* status;
     int* work_counter;  // item counter of the persistent CTAs (zeroed per launch)
     int num_sms;
+    unsigned long long wait_ns;  // limit of every bounded device-side wait
 };
 cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream);
+
+// Failure-path self-test: one CTA waits, with the given limit, on an mbarrier
+// that nothing arrives on (see da2_selftest_wait_timeout in da2.h).
+cudaError_t launch_wait_selftest(unsigned* status, unsigned long long limit_ns, cudaStream_t stream);
+
+// Helpers of the C ABI used by its other translation units.
+int handle_device(const struct ::da2_ctx* h);
+int record_cuda_error(cudaError_t e);
 
 }  // namespace da2

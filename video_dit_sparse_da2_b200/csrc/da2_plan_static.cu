@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "../../include/da2.h"
+#include "da2_kernels.h"
 
 // The working memory (file scope; host code must not pass its name to a
 // kernel: on the host it is only a stand-in, the device address comes from
@@ -27,14 +28,22 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_addr[kMaxDevices] = {};
 
-// Device address of the array on the current device (looked up once).
-int static_scratch(void** out) {
+// Device address of the array on the handle's device, which must be the
+// current device (looked up once per device).
+int static_scratch(da2_handle h, void** out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DA2_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return da2::record_cuda_error(e);
+    if (dev != da2::handle_device(h) || dev < 0 || dev >= kMaxDevices) return DA2_ERR_ARG;
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!g_addr[dev]) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_plan_static) != cudaSuccess || !p) return DA2_ERR_CUDA;
+        e = cudaGetSymbolAddress(&p, g_plan_static);
+        if (e != cudaSuccess) {
+            cudaGetLastError();  // take the error out of the runtime's last-error slot
+            return da2::record_cuda_error(e);
+        }
+        if (!p) return DA2_ERR_CUDA;
         g_addr[dev] = p;
     }
     *out = g_addr[dev];
@@ -51,7 +60,7 @@ extern "C" int da2_plan_static(da2_handle h, const da2_prepared* prep, const da2
     if (rc != DA2_OK) return rc;
     if (sz.plan_scratch > (size_t)DA2_PLAN_STATIC_BYTES) return DA2_ERR_ARG;  // problem too large for the array
     void* scratch = nullptr;
-    if ((rc = static_scratch(&scratch)) != DA2_OK) return rc;
+    if ((rc = static_scratch(h, &scratch)) != DA2_OK) return rc;
     da2_plan_bufs bufs;
     bufs.prec = prec;
     bufs.cnt = cnt;

@@ -20,7 +20,8 @@ OK, ERR_ARG, ERR_ARCH, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4
 # Every symbol include/da2.h declares.
 EXPORTS = ("da2_create", "da2_destroy", "da2_partition", "da2_sizes", "da2_tables", "da2_prepare", "da2_plan",
            "da2_plan_static", "da2_attention",
-           "da2_check_device_status", "da2_status_string", "da2_last_cuda_error")
+           "da2_check_device_status", "da2_set_wait_limit", "da2_selftest_wait_timeout", "da2_status_string",
+           "da2_last_cuda_error")
 
 
 class Shape(ctypes.Structure):
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.da2_attention.argtypes = [P, ctypes.POINTER(PreparedPtrs), ctypes.POINTER(PlanPtrs), P,
                                     ctypes.POINTER(ctypes.c_int64), P]
         L.da2_check_device_status.argtypes = [P, P]
+        L.da2_set_wait_limit.argtypes = [P, ctypes.c_uint64]
+        L.da2_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
         L.da2_status_string.restype = ctypes.c_char_p
         L.da2_status_string.argtypes = [ctypes.c_int]
         L.da2_last_cuda_error.restype = ctypes.c_char_p
@@ -210,6 +213,19 @@ class DA2:
 
     def check_status(self, stream=None):
         _check(lib().da2_check_device_status(self.handle, _stream_ptr(stream)), "device status")
+
+    def status(self, stream=None) -> int:
+        """da2_check_device_status's return code (synchronizes the stream, clears the flag)."""
+        return int(lib().da2_check_device_status(self.handle, _stream_ptr(stream)))
+
+    def set_wait_limit(self, ns: int):
+        """Limit of the kernels' bounded device-side waits (0 = the default 4 s)."""
+        _check(lib().da2_set_wait_limit(self.handle, int(ns)), "da2_set_wait_limit")
+
+    def selftest_wait_timeout(self, ns: int, stream=None):
+        """Enqueue the failure-path self-test kernel (a bounded wait that runs out)."""
+        _check(lib().da2_selftest_wait_timeout(self.handle, int(ns), _stream_ptr(stream)),
+               "da2_selftest_wait_timeout")
 
     def forward(self, q, k, v, bp8, bp4, lam=0.2, out=None, prep=None, plan=None, stream=None, per_row=False):
         """prepare -> plan -> attention; returns (out, prep, plan)."""
