@@ -312,6 +312,19 @@ static inline double bf16_to_double(uint16_t b) {
 
 /* Gather the 64 x d tile of block a of head (b,h) in slot order; padding rows
    are zero. x is [B,H,N,d] bf16 bits, contiguous. */
+/* bf16 of a double, round to nearest even (8 significant bits, the
+   exponent range of float32 with its subnormals).  Used for the weights of
+   the 16-bit path, whose values are at most 1. */
+double oracle_bf16_round(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    frexp(fabs(x), &e); /* |x| in [2^(e-1), 2^e) */
+    int ex = e - 1;
+    if (ex < -126) ex = -126; /* subnormal spacing 2^-133 */
+    double q = ldexp(1.0, ex - 7); /* spacing of the bf16 values near |x| */
+    return nearbyint(x / q) * q;   /* x / q is exact; nearbyint rounds half to even */
+}
+
 static void gather_tile(const o_geom* g, const uint16_t* x, int bh, int a, double* tile) {
     int d = g->d;
     const uint16_t* base = x + (size_t)bh * g->N * d;
@@ -583,15 +596,65 @@ int oracle_assign_rows(int BH, int R, const double* A, int bp8, int bp4, uint8_t
 }
 
 /* ------------------------------------------------------------------------ */
+/* 4c. Three tiers (Table 1's 16-bit share; App. B.6: the 16-bit path takes */
+/* the largest masses, INT8/FP8 the next, NVFP4 the rest).  Cumulative       */
+/* quotas over the ranking of item 4 (per head) or 4b (per row, n = R):      */
+/* C16 = floor(n bp16/10^4), C8 = floor(n (bp16+bp8)/10^4),                  */
+/* Ck = floor(n (bp16+bp8+bp4)/10^4), n = R^2 per head; rank < C16 -> 16,    */
+/* < C8 -> 8, < Ck -> 4, else 0.  With bp16 = 0 this is items 4 / 4b.        */
+/* Lists: 16-bit key blocks ascending, then 8-bit, then 4-bit (the phase     */
+/* order).  cnt i32 [3][BH][R] holds the 8-bit, 4-bit and 16-bit counts.     */
+/* ------------------------------------------------------------------------ */
+int oracle_assign_tiers(int BH, int R, const double* A, int bp16, int bp8, int bp4, int per_row, uint8_t* prec,
+                        int* cnt, uint16_t* kidx) {
+    if (bp16 < 0 || bp8 < 0 || bp4 < 0 || bp16 + bp8 + bp4 > 10000) return -1;
+    long long n = per_row ? (long long)R : (long long)R * R;
+    long long C16 = n * bp16 / 10000, C8 = n * (bp16 + bp8) / 10000, Ck = n * (bp16 + bp8 + bp4) / 10000;
+    size_t BHR = (size_t)BH * R;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < BH; ++bh) {
+        o_pair* pr = (o_pair*)malloc(sizeof(o_pair) * (size_t)n);
+        uint8_t* P = prec + (size_t)bh * R * R;
+        const double* Ah = A + (size_t)bh * R * R;
+        for (int a0 = 0; a0 < (per_row ? R : 1); ++a0) {
+            /* the ranked set: row a0 (per row) or all pairs of the head */
+            size_t base = per_row ? (size_t)a0 * R : 0;
+            for (long long i = 0; i < n; ++i) {
+                pr[i].a = Ah[base + i];
+                pr[i].idx = (int)i;
+            }
+            qsort(pr, (size_t)n, sizeof(o_pair), pair_cmp);
+            for (long long r = 0; r < n; ++r)
+                P[base + pr[r].idx] = (r < C16) ? 16 : (r < C8) ? 8 : (r < Ck) ? 4 : 0;
+        }
+        for (int a = 0; a < R; ++a) {
+            int c[3] = {0, 0, 0}, k = 0;
+            uint16_t* L = kidx + ((size_t)bh * R + a) * R;
+            const uint8_t* Pa = P + (size_t)a * R;
+            for (int b = 0; b < R; ++b) if (Pa[b] == 16) { L[k++] = (uint16_t)b; ++c[2]; }
+            for (int b = 0; b < R; ++b) if (Pa[b] == 8) { L[k++] = (uint16_t)b; ++c[0]; }
+            for (int b = 0; b < R; ++b) if (Pa[b] == 4) { L[k++] = (uint16_t)b; ++c[1]; }
+            for (int t = 0; t < 3; ++t) cnt[t * BHR + (size_t)bh * R + a] = c[t];
+        }
+        free(pr);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* 6. Block-sparse attention with shared normalization (App. B.3, C.1;       */
 /*    Sec. 3.3 phased execution and cross-precision accumulation).           */
 /* For each valid query u of block a, in fp64:                               */
-/*   phases: the 8-bit key blocks of row a (ascending), then the 4-bit ones; */
+/*   phases: the 16-bit key blocks of row a (ascending; only with the tiers  */
+/*   of item 4c), then the 8-bit ones, then the 4-bit ones;                  */
 /*   per key block kb: s_v = (q_u . k_v)/sqrt d with the operands of the     */
 /*   pair's precision, padded keys excluded; m' = max(m, max_v s_v); the     */
 /*   numerator and l are rescaled by e^(m-m'); p_v = e^(s_v - m');           */
 /*   l += sum_v p_v (the unquantized denominator Z^q of App. B.3); the       */
 /*   numerator adds weight_v * valuecode_v.                                  */
+/* 16-bit phase (unit 1): Q, K, V are the bf16 inputs and the weight is      */
+/*   bf16(p_v); entering the 8-bit phase from it the numerator is divided by */
+/*   sigma8 (and by sigma4 when it goes straight to the 4-bit phase).        */
 /* Value codes: 8-bit: e4m3 code of V^T; 4-bit: e2m1 code * ue4m3 group      */
 /*   scale; the tile scale sv[kb] (s8 or g4 of the V tile) is moved into the */
 /*   weight.  Weights and units (reading of the garbled Eq. 8, "entry and    */
@@ -601,7 +664,7 @@ int oracle_assign_rows(int BH, int R, const double* A, int bp8, int bp4, uint8_t
 /*   4-bit phase, unit sigma4 = vmax4/2688: y_v = float(p_v) *               */
 /*     float(sv[kb]/sigma4); per 16 consecutive key slots sf = ue4m3(max y/6)*/
 /*     and weight = e2m1(y_v * (1/sf)) * sf;                                 */
-/*   entering the 4-bit phase the numerator is multiplied by sigma8/sigma4;  */
+/*   entering the 4-bit phase the numerator is multiplied by unit/sigma4;    */
 /*   at the end O = numerator * unit / l, or 0 when no valid key was kept.   */
 /* flags: bit0 quantize Q/K/V; bit1 quantize the weights (needs bit2);       */
 /* bit2 carry the numerator in phase units (production = 7).  Without bit0  */
@@ -609,12 +672,12 @@ int oracle_assign_rows(int BH, int R, const double* A, int bp8, int bp4, uint8_t
 /* the weights are the exact p_v * sv[kb] / unit.                            */
 /* out is f64 [B][H][N][d] in original token order.                          */
 /* ------------------------------------------------------------------------ */
-int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
-                     const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
-                     const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
-                     const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
-                     const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
-                     double* out) {
+static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
+                          const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                          const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
+                          const float* vmax, const int* cnt, int tiers, const uint16_t* kidx, int flags,
+                          const uint8_t* sel, double* out) {
     /* sel: NULL, or one byte per (b,h,block); blocks with sel == 0 are not computed. */
     o_geom g;
     int qops = flags & 1, qw = flags & 2, units = flags & 4;
@@ -629,7 +692,7 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
 #pragma omp parallel for schedule(dynamic)
     for (int bh = 0; bh < BH; ++bh) {
         double* Qt = (double*)malloc(sizeof(double) * tile);
-        double* Qd = (double*)malloc(sizeof(double) * 2 * tile); /* dequantized Q, [phase][slot][c] */
+        double* Qd = (double*)malloc(sizeof(double) * 3 * tile); /* Q per phase (8, 4, 16-bit), [slot][c] */
         double* Kd = (double*)malloc(sizeof(double) * tile);     /* [slot][c] */
         double* Vc = (double*)malloc(sizeof(double) * tile);     /* value codes [slot][c] */
         double* O = (double*)malloc(sizeof(double) * tile);      /* numerators [query slot][c] */
@@ -638,7 +701,7 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
         for (int a = 0; a < R; ++a) {
             size_t ba = (size_t)bh * R + a;
             if (sel && !sel[ba]) continue;
-            int n8 = cnt[ba], n4 = cnt[BHR + ba], nq = g.n_a[a];
+            int n16 = tiers == 3 ? cnt[2 * BHR + ba] : 0, n8 = cnt[ba], n4 = cnt[BHR + ba], nq = g.n_a[a];
             const uint16_t* L = kidx + ba * R;
             gather_tile(&g, q, bh, a, Qt);
             for (int j = 0; j < O_BLOCK; ++j)
@@ -648,6 +711,7 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                     Qd[j * d + c] = qops ? e4[q8[e]] * (double)s8[ba] : x;
                     Qd[tile + j * d + c] =
                         qops ? e2[q4[e]] * e4[sfq[ba * tile / 16 + (size_t)j * G + c / 16]] * (double)g4[ba] : x;
+                    Qd[2 * tile + j * d + c] = x; /* the 16-bit path uses the bf16 operands as they are */
                 }
             /* one softmax state and one numerator per query, shared by both phases */
             for (int u = 0; u < O_BLOCK; ++u) {
@@ -655,15 +719,22 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                 l[u] = 0.0;
             }
             for (size_t i = 0; i < tile; ++i) O[i] = 0.0;
-            double unit = units ? (double)sig8 : 1.0;
-            for (int it = 0; it < n8 + n4; ++it) {
-                int ph = it < n8 ? 0 : 1; /* 0: 8-bit phase, 1: 4-bit phase */
+            /* phases in order: 16-bit (unit 1), 8-bit (unit sigma8), 4-bit (unit sigma4) */
+            double unit = units ? (n16 > 0 ? 1.0 : (double)sig8) : 1.0;
+            for (int it = 0; it < n16 + n8 + n4; ++it) {
+                int ph = it < n16 ? 2 : (it < n16 + n8 ? 0 : 1); /* 0: 8-bit, 1: 4-bit, 2: 16-bit phase */
                 int kb = L[it], nk = g.n_a[kb];
                 size_t bk = (size_t)bh * R + kb;
-                double sv = ph == 0 ? (double)s8[2 * BHR + bk] : (double)g4[2 * BHR + bk];
-                if (it == n8 && units) {
+                double sv = ph == 2 ? 1.0 : (ph == 0 ? (double)s8[2 * BHR + bk] : (double)g4[2 * BHR + bk]);
+                if (units && n16 > 0 && n8 > 0 && it == n16) {
+                    /* Eq. 8, entering the 8-bit phase from the 16-bit one. */
+                    double f = (sig8 > 0.0f) ? unit / (double)sig8 : 1.0;
+                    for (size_t i = 0; i < tile; ++i) O[i] *= f;
+                    unit = (double)sig8;
+                }
+                if (it == n16 + n8 && units) {
                     /* Eq. 8, entering the 4-bit phase: change of numerical units. */
-                    double f = (sig4 > 0.0f) ? (double)sig8 / (double)sig4 : 1.0;
+                    double f = (sig4 > 0.0f) ? unit / (double)sig4 : 1.0;
                     for (size_t i = 0; i < tile; ++i) O[i] *= f;
                     unit = (double)sig4;
                 }
@@ -674,7 +745,9 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                     for (int c = 0; c < d; ++c) {
                         size_t ek = bk * tile + (size_t)j * d + c;
                         size_t ev = bk * tile + (size_t)c * O_BLOCK + j;
-                        if (qops) {
+                        if (qops && ph == 2) {
+                            /* 16-bit: the gathered bf16 values of K and V */
+                        } else if (qops) {
                             Kd[j * d + c] = ph == 0 ? e4[k8[ek]] * (double)s8[BHR + bk]
                                                     : e2[k4[ek]] * e4[sfk[bk * tile / 16 + (size_t)j * G + c / 16]] *
                                                           (double)g4[BHR + bk];
@@ -703,6 +776,8 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                     for (int j = 0; j < nk; ++j) l[u] += p[j];
                     if (!qw) {
                         for (int j = 0; j < O_BLOCK; ++j) w[j] = (unit > 0.0) ? p[j] * sv / unit : 0.0;
+                    } else if (ph == 2) {
+                        for (int j = 0; j < O_BLOCK; ++j) w[j] = oracle_bf16_round(p[j]);
                     } else if (ph == 0) {
                         float ratio = sig8 > 0.0f ? s8[2 * BHR + bk] / sig8 : 0.0f;
                         for (int j = 0; j < O_BLOCK; ++j) w[j] = e4[oracle_e4m3_encode((float)p[j] * ratio)];
@@ -734,6 +809,28 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
     }
     geom_free(&g);
     return 0;
+}
+
+int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                     const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
+                     const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                     const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
+                     const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
+                     double* out) {
+    return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 2,
+                          kidx, flags, sel, out);
+}
+
+/* The same with the 16-bit tier: cnt i32 [3][BH][R] (8-bit, 4-bit, 16-bit
+   counts) and lists holding the 16-bit key blocks first (oracle_assign_tiers). */
+int oracle_attention_tiers(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
+                           const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                           const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
+                           const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
+                           double* out) {
+    return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 3,
+                          kidx, flags, sel, out);
 }
 
 /* Dense softmax attention, for checking the oracle against brute force. */

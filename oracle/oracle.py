@@ -57,6 +57,10 @@ def lib():
         L.oracle_draft.argtypes = [i, i, i, P, ctypes.c_double, P]
         L.oracle_assign.argtypes = [i, i, P, i, i, P, P, P]
         L.oracle_assign_rows.argtypes = [i, i, P, i, i, P, P, P]
+        L.oracle_assign_tiers.argtypes = [i, i, P, i, i, i, i, P, P, P]
+        L.oracle_attention_tiers.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P, P]
+        L.oracle_bf16_round.restype = ctypes.c_double
+        L.oracle_bf16_round.argtypes = [ctypes.c_double]
         L.oracle_attention.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P, P]
         L.oracle_dense.argtypes = [i, i, i, P, P, P, P]
         L.oracle_num_threads.restype = i
@@ -83,6 +87,10 @@ def e2m1_encode(x: float) -> int:
 
 def e2m1_decode(c: int) -> float:
     return float(lib().oracle_e2m1_decode(int(c)))
+
+
+def bf16_round(x: float) -> float:
+    return float(lib().oracle_bf16_round(float(x)))
 
 
 def exp(x: float) -> float:
@@ -181,20 +189,27 @@ def draft(desc: np.ndarray, lam: float = 0.2) -> np.ndarray:
 
 @dataclass
 class Plan:
-    prec: np.ndarray   # u8 [B,H,R,R] in {0,4,8}
-    cnt: np.ndarray    # i32 [2,B,H,R] (8-bit, 4-bit) kept blocks per row
-    kidx: np.ndarray   # u16 [B,H,R,R] row a: 8-bit blocks asc, then 4-bit blocks asc
+    prec: np.ndarray   # u8 [B,H,R,R] in {0,4,8} (and 16 with the 16-bit tier)
+    cnt: np.ndarray    # i32 [2,B,H,R] (8-bit, 4-bit) or [3,B,H,R] (8-bit, 4-bit, 16-bit) kept blocks per row
+    kidx: np.ndarray   # u16 [B,H,R,R] row a: (16-bit blocks asc,) 8-bit blocks asc, then 4-bit blocks asc
 
 
-def assign(A: np.ndarray, bp8: int, bp4: int, per_row: bool = False) -> Plan:
+def assign(A: np.ndarray, bp8: int, bp4: int, per_row: bool = False, bp16: int = 0) -> Plan:
     """Precision of every pair: ranking of all R^2 pairs of a head (the pages),
-    or with per_row of the R key blocks of each query block."""
+    or with per_row of the R key blocks of each query block.  With bp16 > 0
+    the three-tier assignment (cnt gets a third plane, the 16-bit counts)."""
     A = np.ascontiguousarray(A, np.float64)
     B, H, R, _ = A.shape
-    plan = Plan(prec=np.zeros((B, H, R, R), np.uint8), cnt=np.zeros((2, B, H, R), np.int32),
+    tiers = 3 if bp16 else 2
+    plan = Plan(prec=np.zeros((B, H, R, R), np.uint8), cnt=np.zeros((tiers, B, H, R), np.int32),
                 kidx=np.zeros((B, H, R, R), np.uint16))
-    fn = lib().oracle_assign_rows if per_row else lib().oracle_assign
-    if fn(B * H, R, _p(A), int(bp8), int(bp4), _p(plan.prec), _p(plan.cnt), _p(plan.kidx)):
+    if bp16:
+        rc = lib().oracle_assign_tiers(B * H, R, _p(A), int(bp16), int(bp8), int(bp4), int(bool(per_row)),
+                                       _p(plan.prec), _p(plan.cnt), _p(plan.kidx))
+    else:
+        fn = lib().oracle_assign_rows if per_row else lib().oracle_assign
+        rc = fn(B * H, R, _p(A), int(bp8), int(bp4), _p(plan.prec), _p(plan.cnt), _p(plan.kidx))
+    if rc:
         raise ValueError("bad budget")
     return plan
 
@@ -208,7 +223,8 @@ def attention(q, k, v, F, Hv, Wv, prep: Prepared, plan: Plan, flags: int = 7, bl
     B, H, N, d = qb.shape
     out = np.zeros((B, H, N, d), np.float64)
     sel = None if blocks is None else np.ascontiguousarray(blocks, np.uint8)
-    rc = lib().oracle_attention(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(vb), _p(prep.q8), _p(prep.k8),
+    fn = lib().oracle_attention_tiers if plan.cnt.shape[0] == 3 else lib().oracle_attention
+    rc = fn(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(vb), _p(prep.q8), _p(prep.k8),
                                 _p(prep.v8t), _p(prep.s8), _p(prep.q4), _p(prep.k4), _p(prep.v4t),
                                 _p(prep.sfq), _p(prep.sfk), _p(prep.sfv), _p(prep.g4), _p(prep.vmax),
                                 _p(plan.cnt), _p(plan.kidx), int(flags),
@@ -226,10 +242,10 @@ def dense(q, k, v) -> np.ndarray:
     return out
 
 
-def run(q, k, v, F, Hv, Wv, bp8, bp4, lam=0.2, flags=7, per_row=False):
+def run(q, k, v, F, Hv, Wv, bp8, bp4, lam=0.2, flags=7, per_row=False, bp16=0):
     """Whole pipeline: prepare -> draft -> assign -> attention."""
     prep = prepare(q, k, v, F, Hv, Wv)
     A = draft(prep.desc, lam)
-    plan = assign(A, bp8, bp4, per_row)
+    plan = assign(A, bp8, bp4, per_row, bp16)
     out = attention(q, k, v, F, Hv, Wv, prep, plan, flags)
     return prep, A, plan, out
