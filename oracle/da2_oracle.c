@@ -473,6 +473,54 @@ int oracle_prepare(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q
 }
 
 /* ------------------------------------------------------------------------ */
+/* 5b. INT8 operands of the paper's 8-bit QK^T (App. C.1: "The INT8 path    */
+/* uses INT8 for QK^T and FP8 for the probability-value multiplication";    */
+/* the scale placement is a reading, as for FP8): per 64-token tile         */
+/* s = amax/127 (fp32 divide), code = clamp(RNE(x * (127/amax)), -127, 127) */
+/* with the product rounded in fp32; dequantized value = code * s; a zero   */
+/* tile has s = 0 and all-zero codes.                                        */
+/*   q8i,k8i s8 [B][H][R][64][d]; si8 f32 [2][B][H][R] (Q, K)                */
+/* ------------------------------------------------------------------------ */
+int8_t oracle_int8_encode(float x) {
+    float r = nearbyintf(x); /* round half to even */
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+int oracle_prepare_int8(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                        int8_t* q8i, int8_t* k8i, float* si8) {
+    o_geom g;
+    if (d % 16 || geom_make(&g, B, H, d, F, Hv, Wv)) return -1;
+    int R = g.R, BH = B * H;
+    size_t tile = (size_t)O_BLOCK * d;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < BH; ++bh) {
+        double* t = (double*)malloc(sizeof(double) * tile);
+        for (int a = 0; a < R; ++a) {
+            size_t ba = (size_t)bh * R + a;
+            for (int which = 0; which < 2; ++which) {
+                gather_tile(&g, which == 0 ? q : k, bh, a, t);
+                float amax = tile_amax(t, (int)tile);
+                int8_t* c = (which == 0 ? q8i : k8i) + ba * tile;
+                float* sc = si8 + (size_t)which * BH * R + ba;
+                if (amax == 0.0f) {
+                    *sc = 0.0f;
+                    memset(c, 0, tile);
+                    continue;
+                }
+                *sc = amax / 127.0f;
+                float inv = 127.0f / amax;
+                for (size_t i = 0; i < tile; ++i) c[i] = oracle_int8_encode((float)t[i] * inv);
+            }
+        }
+        free(t);
+    }
+    geom_free(&g);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* 3. Draft map (Eq. 3; App. C.1: both branches normalize over key regions). */
 /* logit = (sum_c q_c k_c, as an fma chain in ascending c from 0) * (1/sqrt d);*/
 /* row softmax with m = row max, e_b = o_exp(l_b - m), Z = sum_b e_b in       */
@@ -667,6 +715,7 @@ int oracle_assign_tiers(int BH, int R, const double* A, int bp16, int bp8, int b
 /*   entering the 4-bit phase the numerator is multiplied by unit/sigma4;    */
 /*   at the end O = numerator * unit / l, or 0 when no valid key was kept.   */
 /* flags: bit0 quantize Q/K/V; bit1 quantize the weights (needs bit2);       */
+/* bit3 (with the operands of item 5b) the 8-bit phase's QK^T in INT8;       */
 /* bit2 carry the numerator in phase units (production = 7).  Without bit0  */
 /* the value "codes" are the exact values divided by sv[kb]; without bit1    */
 /* the weights are the exact p_v * sv[kb] / unit.                            */
@@ -677,10 +726,12 @@ static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, const uint
                           const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
                           const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
                           const float* vmax, const int* cnt, int tiers, const uint16_t* kidx, int flags,
-                          const uint8_t* sel, double* out) {
+                          const uint8_t* sel, const int8_t* q8i, const int8_t* k8i, const float* si8,
+                          double* out) {
     /* sel: NULL, or one byte per (b,h,block); blocks with sel == 0 are not computed. */
     o_geom g;
     int qops = flags & 1, qw = flags & 2, units = flags & 4;
+    int i8 = (flags & 8) && q8i && k8i && si8; /* the 8-bit phase's QK^T in INT8 */
     if (qw && !units) return -2;
     if (geom_make(&g, B, H, d, F, Hv, Wv)) return -1;
     int R = g.R, BH = B * H, N = g.N, G = d / 16;
@@ -708,7 +759,7 @@ static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, const uint
                 for (int c = 0; c < d; ++c) {
                     size_t e = ba * tile + (size_t)j * d + c;
                     double x = Qt[j * d + c];
-                    Qd[j * d + c] = qops ? e4[q8[e]] * (double)s8[ba] : x;
+                    Qd[j * d + c] = qops ? (i8 ? (double)q8i[e] * (double)si8[ba] : e4[q8[e]] * (double)s8[ba]) : x;
                     Qd[tile + j * d + c] =
                         qops ? e2[q4[e]] * e4[sfq[ba * tile / 16 + (size_t)j * G + c / 16]] * (double)g4[ba] : x;
                     Qd[2 * tile + j * d + c] = x; /* the 16-bit path uses the bf16 operands as they are */
@@ -748,7 +799,8 @@ static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, const uint
                         if (qops && ph == 2) {
                             /* 16-bit: the gathered bf16 values of K and V */
                         } else if (qops) {
-                            Kd[j * d + c] = ph == 0 ? e4[k8[ek]] * (double)s8[BHR + bk]
+                            Kd[j * d + c] = ph == 0 ? (i8 ? (double)k8i[ek] * (double)si8[BHR + bk]
+                                                          : e4[k8[ek]] * (double)s8[BHR + bk])
                                                     : e2[k4[ek]] * e4[sfk[bk * tile / 16 + (size_t)j * G + c / 16]] *
                                                           (double)g4[BHR + bk];
                             Vc[j * d + c] = ph == 0 ? e4[v8t[ev]]
@@ -818,7 +870,7 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                      const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
                      double* out) {
     return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 2,
-                          kidx, flags, sel, out);
+                          kidx, flags, sel, NULL, NULL, NULL, out);
 }
 
 /* The same with the 16-bit tier: cnt i32 [3][BH][R] (8-bit, 4-bit, 16-bit
@@ -830,7 +882,20 @@ int oracle_attention_tiers(int B, int H, int d, int F, int Hv, int Wv, const uin
                            const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
                            double* out) {
     return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 3,
-                          kidx, flags, sel, out);
+                          kidx, flags, sel, NULL, NULL, NULL, out);
+}
+
+/* Either tier layout (tiers = 2 or 3) with the 8-bit phase's QK^T in INT8
+   (flags bit 3, item 5b operands; FP8 PV as before). */
+int oracle_attention_int8(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                          const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
+                          const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                          const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
+                          const float* vmax, const int* cnt, int tiers, const uint16_t* kidx, int flags,
+                          const uint8_t* sel, const int8_t* q8i, const int8_t* k8i, const float* si8, double* out) {
+    if (tiers != 2 && tiers != 3) return -1;
+    return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt,
+                          tiers, kidx, flags | 8, sel, q8i, k8i, si8, out);
 }
 
 /* Dense softmax attention, for checking the oracle against brute force. */

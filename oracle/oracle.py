@@ -59,6 +59,10 @@ def lib():
         L.oracle_assign_rows.argtypes = [i, i, P, i, i, P, P, P]
         L.oracle_assign_tiers.argtypes = [i, i, P, i, i, i, i, P, P, P]
         L.oracle_attention_tiers.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P, P]
+        L.oracle_int8_encode.restype = ctypes.c_int8
+        L.oracle_int8_encode.argtypes = [ctypes.c_float]
+        L.oracle_prepare_int8.argtypes = [i] * 6 + [P] * 5
+        L.oracle_attention_int8.argtypes = [i] * 6 + [P] * 3 + [P] * 13 + [i, P, i, P, P, P, P, P]
         L.oracle_bf16_round.restype = ctypes.c_double
         L.oracle_bf16_round.argtypes = [ctypes.c_double]
         L.oracle_attention.argtypes = [i] * 6 + [P] * 3 + [P] * 14 + [i, P, P]
@@ -87,6 +91,23 @@ def e2m1_encode(x: float) -> int:
 
 def e2m1_decode(c: int) -> float:
     return float(lib().oracle_e2m1_decode(int(c)))
+
+
+def int8_encode(x: float) -> int:
+    return int(lib().oracle_int8_encode(float(x)))
+
+
+def prepare_int8(q, k, F: int, Hv: int, Wv: int):
+    """INT8 tiles of Q and K (s8 [B,H,R,64,d] each) and their tile scales f32 [2,B,H,R]."""
+    qb, kb = _bits(q), _bits(k)
+    B, H, N, d = qb.shape
+    R = F * (-(-(Hv * Wv) // BLOCK))
+    q8i = np.zeros((B, H, R, BLOCK, d), np.int8)
+    k8i = np.zeros((B, H, R, BLOCK, d), np.int8)
+    si8 = np.zeros((2, B, H, R), np.float32)
+    if lib().oracle_prepare_int8(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(q8i), _p(k8i), _p(si8)):
+        raise ValueError("oracle_prepare_int8 failed")
+    return q8i, k8i, si8
 
 
 def bf16_round(x: float) -> float:
@@ -214,15 +235,26 @@ def assign(A: np.ndarray, bp8: int, bp4: int, per_row: bool = False, bp16: int =
     return plan
 
 
-def attention(q, k, v, F, Hv, Wv, prep: Prepared, plan: Plan, flags: int = 7, blocks=None) -> np.ndarray:
+def attention(q, k, v, F, Hv, Wv, prep: Prepared, plan: Plan, flags: int = 7, blocks=None, int8=None) -> np.ndarray:
     """Block-sparse mixed-precision attention, f64 [B,H,N,d] in token order.
 
     blocks: optional boolean [B,H,R] selecting the query blocks to compute
-    (the other tokens stay 0)."""
+    (the other tokens stay 0).  int8: optional (q8i, k8i, si8) of
+    prepare_int8, for the 8-bit phase's QK^T in INT8."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, H, N, d = qb.shape
     out = np.zeros((B, H, N, d), np.float64)
     sel = None if blocks is None else np.ascontiguousarray(blocks, np.uint8)
+    if int8 is not None:
+        q8i, k8i, si8 = (np.ascontiguousarray(x) for x in int8)
+        rc = lib().oracle_attention_int8(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(vb), _p(prep.q8), _p(prep.k8),
+                                         _p(prep.v8t), _p(prep.s8), _p(prep.q4), _p(prep.k4), _p(prep.v4t),
+                                         _p(prep.sfq), _p(prep.sfk), _p(prep.sfv), _p(prep.g4), _p(prep.vmax),
+                                         _p(plan.cnt), int(plan.cnt.shape[0]), _p(plan.kidx), int(flags),
+                                         None if sel is None else _p(sel), _p(q8i), _p(k8i), _p(si8), _p(out))
+        if rc:
+            raise ValueError(f"oracle_attention_int8 failed ({rc})")
+        return out
     fn = lib().oracle_attention_tiers if plan.cnt.shape[0] == 3 else lib().oracle_attention
     rc = fn(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(vb), _p(prep.q8), _p(prep.k8),
                                 _p(prep.v8t), _p(prep.s8), _p(prep.q4), _p(prep.k4), _p(prep.v4t),
@@ -242,10 +274,11 @@ def dense(q, k, v) -> np.ndarray:
     return out
 
 
-def run(q, k, v, F, Hv, Wv, bp8, bp4, lam=0.2, flags=7, per_row=False, bp16=0):
-    """Whole pipeline: prepare -> draft -> assign -> attention."""
+def run(q, k, v, F, Hv, Wv, bp8, bp4, lam=0.2, flags=7, per_row=False, bp16=0, int8=False):
+    """Whole pipeline: prepare -> draft -> assign -> attention (int8: the
+    8-bit phase's QK^T in INT8)."""
     prep = prepare(q, k, v, F, Hv, Wv)
     A = draft(prep.desc, lam)
     plan = assign(A, bp8, bp4, per_row, bp16)
-    out = attention(q, k, v, F, Hv, Wv, prep, plan, flags)
+    out = attention(q, k, v, F, Hv, Wv, prep, plan, flags, int8=prepare_int8(q, k, F, Hv, Wv) if int8 else None)
     return prep, A, plan, out
