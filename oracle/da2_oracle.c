@@ -260,22 +260,30 @@ int oracle_partition(int Hv, int Wv, int C, int* region_of, int* slot_of, int* n
 /* ------------------------------------------------------------------------ */
 /* Shapes and the token <-> slot tables.                                     */
 /* ------------------------------------------------------------------------ */
+/* Prefix (text) tokens, App. C.1 ("Prefix interactions lie outside the     */
+/* video-region budget").  Reading of the sequence layout, which the pages  */
+/* do not give: the P prefix tokens come first (positions 0..P-1), the      */
+/* video tokens follow in raster order (P + f*Hv*Wv + y*Wv + x).  The       */
+/* prefix is packed into Rp = ceil(P/64) blocks of consecutive tokens, which */
+/* follow the Rv video blocks: block Rv + i holds tokens 64i .. 64i+63.     */
 typedef struct {
-    int B, H, d, F, Hv, Wv;
-    int Rf, R, N, Npad;
+    int B, H, d, F, Hv, Wv, P;
+    int Rf, Rv, Rp, R, N, Npad; /* R = Rv + Rp blocks */
     int* slot_token; /* [Npad] token index of packed slot, -1 for padding */
     int* n_a;        /* [R] valid tokens of region (block) a */
 } o_geom;
 
-static int geom_make(o_geom* g, int B, int H, int d, int F, int Hv, int Wv) {
-    g->B = B; g->H = H; g->d = d; g->F = F; g->Hv = Hv; g->Wv = Wv;
+static int geom_make_p(o_geom* g, int B, int H, int d, int F, int Hv, int Wv, int P) {
+    if (P < 0) return -1;
+    g->B = B; g->H = H; g->d = d; g->F = F; g->Hv = Hv; g->Wv = Wv; g->P = P;
     int n = Hv * Wv;
     int* region_of = (int*)malloc(sizeof(int) * n);
     int* slot_of = (int*)malloc(sizeof(int) * n);
     int* nf = (int*)malloc(sizeof(int) * n);
     int Rf = oracle_partition(Hv, Wv, O_BLOCK, region_of, slot_of, nf);
     if (Rf <= 0) { free(region_of); free(slot_of); free(nf); return -1; }
-    g->Rf = Rf; g->R = F * Rf; g->N = F * n; g->Npad = g->R * O_BLOCK;
+    g->Rf = Rf; g->Rv = F * Rf; g->Rp = (P + O_BLOCK - 1) / O_BLOCK; g->R = g->Rv + g->Rp;
+    g->N = P + F * n; g->Npad = g->R * O_BLOCK;
     g->slot_token = (int*)malloc(sizeof(int) * g->Npad);
     g->n_a = (int*)malloc(sizeof(int) * g->R);
     for (int i = 0; i < g->Npad; ++i) g->slot_token[i] = -1;
@@ -283,14 +291,35 @@ static int geom_make(o_geom* g, int B, int H, int d, int F, int Hv, int Wv) {
         for (int j = 0; j < Rf; ++j) g->n_a[f * Rf + j] = nf[j];
         for (int c = 0; c < n; ++c) {
             int a = f * Rf + region_of[c];
-            g->slot_token[a * O_BLOCK + slot_of[c]] = f * n + c;
+            g->slot_token[a * O_BLOCK + slot_of[c]] = P + f * n + c;
         }
+    }
+    for (int i = 0; i < g->Rp; ++i) {
+        int a = g->Rv + i, cnt = P - i * O_BLOCK < O_BLOCK ? P - i * O_BLOCK : O_BLOCK;
+        g->n_a[a] = cnt;
+        for (int s2 = 0; s2 < cnt; ++s2) g->slot_token[a * O_BLOCK + s2] = i * O_BLOCK + s2;
     }
     free(region_of); free(slot_of); free(nf);
     return 0;
 }
 
+static int geom_make(o_geom* g, int B, int H, int d, int F, int Hv, int Wv) {
+    return geom_make_p(g, B, H, d, F, Hv, Wv, 0);
+}
+
 static void geom_free(o_geom* g) { free(g->slot_token); free(g->n_a); }
+
+/* Packed-slot -> token table for a shape with P prefix tokens; returns the
+   number of blocks (video, then prefix), or -1. */
+int oracle_slot_tokens_p(int F, int Hv, int Wv, int P, int* slot_token, int* n_a) {
+    o_geom g;
+    if (geom_make_p(&g, 1, 1, 64, F, Hv, Wv, P)) return -1;
+    memcpy(slot_token, g.slot_token, sizeof(int) * g.Npad);
+    memcpy(n_a, g.n_a, sizeof(int) * g.R);
+    int R = g.R;
+    geom_free(&g);
+    return R;
+}
 
 /* Packed-slot -> token table for a shape; returns R, or -1. */
 int oracle_slot_tokens(int F, int Hv, int Wv, int* slot_token, int* n_a) {
@@ -390,12 +419,15 @@ static void quant_fp4_group(const float* v16, float amax, float g, uint8_t* code
  *   g4       f32 [3][B][H][R]        NVFP4 tile scales of Q, K, V
  *   vmax     f32 [2][B][H]           max_kb s8_V[kb], max_kb g4_V[kb]
  */
-int oracle_prepare(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
-                   const uint16_t* v, double* desc, uint8_t* q8, uint8_t* k8, uint8_t* v8t, float* s8,
-                   uint8_t* q4, uint8_t* k4, uint8_t* v4t, uint8_t* sfq, uint8_t* sfk, uint8_t* sfv,
-                   float* g4, float* vmax) {
+/* With P prefix tokens every block (video, then prefix) is prepared; the V
+   maxima (the units of the 8-bit and 4-bit phases, which only video pairs
+   use) are taken over the video blocks. */
+int oracle_prepare_p(int B, int H, int d, int F, int Hv, int Wv, int P, const uint16_t* q, const uint16_t* k,
+                     const uint16_t* v, double* desc, uint8_t* q8, uint8_t* k8, uint8_t* v8t, float* s8,
+                     uint8_t* q4, uint8_t* k4, uint8_t* v4t, uint8_t* sfq, uint8_t* sfk, uint8_t* sfv,
+                     float* g4, float* vmax) {
     o_geom g;
-    if (d % 16 || geom_make(&g, B, H, d, F, Hv, Wv)) return -1;
+    if (d % 16 || geom_make_p(&g, B, H, d, F, Hv, Wv, P)) return -1;
     int R = g.R, BH = B * H;
     size_t tile = (size_t)O_BLOCK * d;
 #pragma omp parallel for schedule(dynamic)
@@ -459,8 +491,10 @@ int oracle_prepare(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q
                             for (int i = 0; i < 16; ++i) f16[i] = (float)tt[c * O_BLOCK + gi * 16 + i];
                             quant_fp4_group(f16, amax, gt, c4 + c * O_BLOCK + gi * 16, sf + c * 4 + gi);
                         }
-                    vm8 = fmaxf(vm8, s8[(size_t)2 * BH * R + ba]);
-                    vm4 = fmaxf(vm4, gt);
+                    if (a < g.Rv) {
+                        vm8 = fmaxf(vm8, s8[(size_t)2 * BH * R + ba]);
+                        vm4 = fmaxf(vm4, gt);
+                    }
                 }
             }
         }
@@ -470,6 +504,14 @@ int oracle_prepare(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q
     }
     geom_free(&g);
     return 0;
+}
+
+int oracle_prepare(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                   const uint16_t* v, double* desc, uint8_t* q8, uint8_t* k8, uint8_t* v8t, float* s8,
+                   uint8_t* q4, uint8_t* k4, uint8_t* v4t, uint8_t* sfq, uint8_t* sfk, uint8_t* sfv,
+                   float* g4, float* vmax) {
+    return oracle_prepare_p(B, H, d, F, Hv, Wv, 0, q, k, v, desc, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4,
+                            vmax);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -488,10 +530,10 @@ int8_t oracle_int8_encode(float x) {
     return (int8_t)r;
 }
 
-int oracle_prepare_int8(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
-                        int8_t* q8i, int8_t* k8i, float* si8) {
+int oracle_prepare_int8_p(int B, int H, int d, int F, int Hv, int Wv, int P, const uint16_t* q, const uint16_t* k,
+                          int8_t* q8i, int8_t* k8i, float* si8) {
     o_geom g;
-    if (d % 16 || geom_make(&g, B, H, d, F, Hv, Wv)) return -1;
+    if (d % 16 || geom_make_p(&g, B, H, d, F, Hv, Wv, P)) return -1;
     int R = g.R, BH = B * H;
     size_t tile = (size_t)O_BLOCK * d;
 #pragma omp parallel for schedule(dynamic)
@@ -518,6 +560,11 @@ int oracle_prepare_int8(int B, int H, int d, int F, int Hv, int Wv, const uint16
     }
     geom_free(&g);
     return 0;
+}
+
+int oracle_prepare_int8(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+                        int8_t* q8i, int8_t* k8i, float* si8) {
+    return oracle_prepare_int8_p(B, H, d, F, Hv, Wv, 0, q, k, q8i, k8i, si8);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -690,6 +737,49 @@ int oracle_assign_tiers(int BH, int R, const double* A, int bp16, int bp8, int b
 }
 
 /* ------------------------------------------------------------------------ */
+/* 4d. Prefix keys and queries (App. C.1: "video queries retain all valid    */
+/* prefix keys, and prefix queries use non-sparse attention"; "Prefix        */
+/* interactions lie outside the video-region budget").  Reading of the      */
+/* unstated precision: both run on the 16-bit path, the reference precision */
+/* (the budget that assigns the lower precisions covers only video-region   */
+/* pairs).  From a video plan (cnt [3][BH][Rv], lists [BH][Rv][Rv] of item  */
+/* 4c, 16-bit blocks first) build the plan over all Rt = Rv + Rp blocks: a  */
+/* video row gets the prefix blocks Rv..Rt-1 after its 16-bit video blocks  */
+/* (ascending block order within the phase); a prefix row gets every block  */
+/* 0..Rt-1 at 16 bits.  cnt_t [3][BH][Rt], kidx_t [BH][Rt][Rt].              */
+/* ------------------------------------------------------------------------ */
+int oracle_prefix_plan(int BH, int Rv, int Rp, const int* cnt_v, const uint16_t* kidx_v, int* cnt_t,
+                       uint16_t* kidx_t) {
+    if (BH <= 0 || Rv <= 0 || Rp < 0) return -1;
+    int Rt = Rv + Rp;
+    size_t BHRv = (size_t)BH * Rv, BHRt = (size_t)BH * Rt;
+    for (int bh = 0; bh < BH; ++bh) {
+        for (int a = 0; a < Rt; ++a) {
+            size_t rt = (size_t)bh * Rt + a;
+            uint16_t* L = kidx_t + rt * Rt;
+            if (a < Rv) {
+                size_t rv = (size_t)bh * Rv + a;
+                int n8 = cnt_v[rv], n4 = cnt_v[BHRv + rv], n16 = cnt_v[2 * BHRv + rv];
+                const uint16_t* Lv = kidx_v + rv * Rv;
+                int k = 0;
+                for (int i = 0; i < n16; ++i) L[k++] = Lv[i];
+                for (int i = 0; i < Rp; ++i) L[k++] = (uint16_t)(Rv + i);
+                for (int i = n16; i < n16 + n8 + n4; ++i) L[k++] = Lv[i];
+                cnt_t[rt] = n8;
+                cnt_t[BHRt + rt] = n4;
+                cnt_t[2 * BHRt + rt] = n16 + Rp;
+            } else {
+                for (int b = 0; b < Rt; ++b) L[b] = (uint16_t)b;
+                cnt_t[rt] = 0;
+                cnt_t[BHRt + rt] = 0;
+                cnt_t[2 * BHRt + rt] = Rt;
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* 6. Block-sparse attention with shared normalization (App. B.3, C.1;       */
 /*    Sec. 3.3 phased execution and cross-precision accumulation).           */
 /* For each valid query u of block a, in fp64:                               */
@@ -721,7 +811,7 @@ int oracle_assign_tiers(int BH, int R, const double* A, int bp16, int bp8, int b
 /* the weights are the exact p_v * sv[kb] / unit.                            */
 /* out is f64 [B][H][N][d] in original token order.                          */
 /* ------------------------------------------------------------------------ */
-static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q, const uint16_t* k,
+static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, int P, const uint16_t* q, const uint16_t* k,
                           const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
                           const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
                           const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
@@ -733,7 +823,7 @@ static int attention_impl(int B, int H, int d, int F, int Hv, int Wv, const uint
     int qops = flags & 1, qw = flags & 2, units = flags & 4;
     int i8 = (flags & 8) && q8i && k8i && si8; /* the 8-bit phase's QK^T in INT8 */
     if (qw && !units) return -2;
-    if (geom_make(&g, B, H, d, F, Hv, Wv)) return -1;
+    if (geom_make_p(&g, B, H, d, F, Hv, Wv, P)) return -1;
     int R = g.R, BH = B * H, N = g.N, G = d / 16;
     size_t tile = (size_t)O_BLOCK * d, BHR = (size_t)BH * R;
     double rd = 1.0 / sqrt((double)d);
@@ -869,7 +959,7 @@ int oracle_attention(int B, int H, int d, int F, int Hv, int Wv, const uint16_t*
                      const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
                      const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
                      double* out) {
-    return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 2,
+    return attention_impl(B, H, d, F, Hv, Wv, 0, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 2,
                           kidx, flags, sel, NULL, NULL, NULL, out);
 }
 
@@ -881,7 +971,7 @@ int oracle_attention_tiers(int B, int H, int d, int F, int Hv, int Wv, const uin
                            const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
                            const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
                            double* out) {
-    return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 3,
+    return attention_impl(B, H, d, F, Hv, Wv, 0, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt, 3,
                           kidx, flags, sel, NULL, NULL, NULL, out);
 }
 
@@ -894,8 +984,22 @@ int oracle_attention_int8(int B, int H, int d, int F, int Hv, int Wv, const uint
                           const float* vmax, const int* cnt, int tiers, const uint16_t* kidx, int flags,
                           const uint8_t* sel, const int8_t* q8i, const int8_t* k8i, const float* si8, double* out) {
     if (tiers != 2 && tiers != 3) return -1;
-    return attention_impl(B, H, d, F, Hv, Wv, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt,
+    return attention_impl(B, H, d, F, Hv, Wv, 0, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt,
                           tiers, kidx, flags | 8, sel, q8i, k8i, si8, out);
+}
+
+/* The attention with P prefix tokens: operands of all Rt blocks (video,
+   then prefix; oracle_prepare_p), the three-tier plan over Rt blocks
+   (oracle_prefix_plan) and, optionally (q8i non-null), the INT8 operands of
+   the 8-bit phase's QK^T.  out f64 [B][H][P + F*Hv*Wv][d] in token order. */
+int oracle_attention_p(int B, int H, int d, int F, int Hv, int Wv, int P, const uint16_t* q, const uint16_t* k,
+                       const uint16_t* v, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
+                       const float* s8, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                       const uint8_t* sfq, const uint8_t* sfk, const uint8_t* sfv, const float* g4,
+                       const float* vmax, const int* cnt, const uint16_t* kidx, int flags, const uint8_t* sel,
+                       const int8_t* q8i, const int8_t* k8i, const float* si8, double* out) {
+    return attention_impl(B, H, d, F, Hv, Wv, P, q, k, v, q8, k8, v8t, s8, q4, k4, v4t, sfq, sfk, sfv, g4, vmax, cnt,
+                          3, kidx, q8i ? (flags | 8) : flags, sel, q8i, k8i, si8, out);
 }
 
 /* Dense softmax attention, for checking the oracle against brute force. */

@@ -62,6 +62,11 @@ def lib():
         L.oracle_int8_encode.restype = ctypes.c_int8
         L.oracle_int8_encode.argtypes = [ctypes.c_float]
         L.oracle_prepare_int8.argtypes = [i] * 6 + [P] * 5
+        L.oracle_prepare_int8_p.argtypes = [i] * 7 + [P] * 5
+        L.oracle_prepare_p.argtypes = [i] * 7 + [P] * 3 + [P] * 13
+        L.oracle_slot_tokens_p.argtypes = [i, i, i, i, P, P]
+        L.oracle_prefix_plan.argtypes = [i, i, i, P, P, P, P]
+        L.oracle_attention_p.argtypes = [i] * 7 + [P] * 3 + [P] * 14 + [i, P, P, P, P, P]
         L.oracle_attention_int8.argtypes = [i] * 6 + [P] * 3 + [P] * 13 + [i, P, i, P, P, P, P, P]
         L.oracle_bf16_round.restype = ctypes.c_double
         L.oracle_bf16_round.argtypes = [ctypes.c_double]
@@ -97,15 +102,15 @@ def int8_encode(x: float) -> int:
     return int(lib().oracle_int8_encode(float(x)))
 
 
-def prepare_int8(q, k, F: int, Hv: int, Wv: int):
+def prepare_int8(q, k, F: int, Hv: int, Wv: int, P: int = 0):
     """INT8 tiles of Q and K (s8 [B,H,R,64,d] each) and their tile scales f32 [2,B,H,R]."""
     qb, kb = _bits(q), _bits(k)
     B, H, N, d = qb.shape
-    R = F * (-(-(Hv * Wv) // BLOCK))
+    R = F * (-(-(Hv * Wv) // BLOCK)) + -(-P // BLOCK)
     q8i = np.zeros((B, H, R, BLOCK, d), np.int8)
     k8i = np.zeros((B, H, R, BLOCK, d), np.int8)
     si8 = np.zeros((2, B, H, R), np.float32)
-    if lib().oracle_prepare_int8(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(q8i), _p(k8i), _p(si8)):
+    if lib().oracle_prepare_int8_p(B, H, d, F, Hv, Wv, int(P), _p(qb), _p(kb), _p(q8i), _p(k8i), _p(si8)):
         raise ValueError("oracle_prepare_int8 failed")
     return q8i, k8i, si8
 
@@ -134,14 +139,15 @@ def partition(Hv: int, Wv: int, C: int = BLOCK):
     return region_of, slot_of, n_a[:Rf].copy()
 
 
-def slot_tokens(F: int, Hv: int, Wv: int):
-    """Token index held by each packed slot (-1 = padding) and valid counts per block."""
+def slot_tokens(F: int, Hv: int, Wv: int, P: int = 0):
+    """Token index held by each packed slot (-1 = padding) and valid counts per
+    block; with P prefix tokens the prefix blocks follow the video blocks."""
     n = Hv * Wv
     Rf = -(-n // BLOCK)
-    R = F * Rf
+    R = F * Rf + -(-P // BLOCK)
     st = np.zeros(R * BLOCK, np.int32)
     na = np.zeros(R, np.int32)
-    if lib().oracle_slot_tokens(F, Hv, Wv, _p(st), _p(na)) != R:
+    if lib().oracle_slot_tokens_p(F, Hv, Wv, int(P), _p(st), _p(na)) != R:
         raise ValueError("bad shape")
     return st, na
 
@@ -177,11 +183,13 @@ def _bits(x) -> np.ndarray:
     return x
 
 
-def prepare(q, k, v, F: int, Hv: int, Wv: int) -> Prepared:
+def prepare(q, k, v, F: int, Hv: int, Wv: int, P: int = 0) -> Prepared:
+    """Prepared operands of every block: the video blocks, then (P > 0) the
+    prefix blocks."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, H, N, d = qb.shape
-    R = F * (-(-(Hv * Wv) // BLOCK))
-    assert N == F * Hv * Wv
+    R = F * (-(-(Hv * Wv) // BLOCK)) + -(-P // BLOCK)
+    assert N == P + F * Hv * Wv
     out = Prepared(
         desc=np.zeros((4, B, H, R, d), np.float64),
         q8=np.zeros((B, H, R, BLOCK, d), np.uint8), k8=np.zeros((B, H, R, BLOCK, d), np.uint8),
@@ -191,7 +199,7 @@ def prepare(q, k, v, F: int, Hv: int, Wv: int) -> Prepared:
         sfq=np.zeros((B, H, R, BLOCK, d // 16), np.uint8), sfk=np.zeros((B, H, R, BLOCK, d // 16), np.uint8),
         sfv=np.zeros((B, H, R, d, 4), np.uint8), g4=np.zeros((3, B, H, R), np.float32),
         vmax=np.zeros((2, B, H), np.float32))
-    rc = lib().oracle_prepare(B, H, d, F, Hv, Wv, _p(qb), _p(kb), _p(vb), _p(out.desc), _p(out.q8), _p(out.k8),
+    rc = lib().oracle_prepare_p(B, H, d, F, Hv, Wv, int(P), _p(qb), _p(kb), _p(vb), _p(out.desc), _p(out.q8), _p(out.k8),
                               _p(out.v8t), _p(out.s8), _p(out.q4), _p(out.k4), _p(out.v4t), _p(out.sfq),
                               _p(out.sfk), _p(out.sfv), _p(out.g4), _p(out.vmax))
     if rc:
@@ -233,6 +241,62 @@ def assign(A: np.ndarray, bp8: int, bp4: int, per_row: bool = False, bp16: int =
     if rc:
         raise ValueError("bad budget")
     return plan
+
+
+def prefix_plan(plan: Plan, Rp: int) -> Plan:
+    """The plan over the video and the Rp prefix blocks (App. C.1 prefix rule,
+    reading in da2_oracle.c item 4d) from a three-plane video plan."""
+    assert plan.cnt.shape[0] == 3, "needs the three-tier plan (assign with bp16, or tiers_plan)"
+    _, B, H, Rv = plan.cnt.shape
+    Rt = Rv + Rp
+    out = Plan(prec=plan.prec, cnt=np.zeros((3, B, H, Rt), np.int32), kidx=np.zeros((B, H, Rt, Rt), np.uint16))
+    if lib().oracle_prefix_plan(B * H, Rv, Rp, _p(np.ascontiguousarray(plan.cnt)),
+                                _p(np.ascontiguousarray(plan.kidx)), _p(out.cnt), _p(out.kidx)):
+        raise ValueError("oracle_prefix_plan failed")
+    return out
+
+
+def tiers_plan(A: np.ndarray, bp8: int, bp4: int, per_row: bool = False, bp16: int = 0) -> Plan:
+    """The three-plane (three-tier) plan, also when bp16 = 0."""
+    A = np.ascontiguousarray(A, np.float64)
+    B, H, R, _ = A.shape
+    plan = Plan(prec=np.zeros((B, H, R, R), np.uint8), cnt=np.zeros((3, B, H, R), np.int32),
+                kidx=np.zeros((B, H, R, R), np.uint16))
+    if lib().oracle_assign_tiers(B * H, R, _p(A), int(bp16), int(bp8), int(bp4), int(bool(per_row)),
+                                 _p(plan.prec), _p(plan.cnt), _p(plan.kidx)):
+        raise ValueError("bad budget")
+    return plan
+
+
+def attention_prefix(q, k, v, F, Hv, Wv, P, prep: Prepared, plan: Plan, flags: int = 7, blocks=None,
+                     int8=None) -> np.ndarray:
+    """Attention with P prefix tokens (plan from prefix_plan), f64 [B,H,N,d]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, N, d = qb.shape
+    out = np.zeros((B, H, N, d), np.float64)
+    sel = None if blocks is None else np.ascontiguousarray(blocks, np.uint8)
+    q8i, k8i, si8 = (None, None, None) if int8 is None else (np.ascontiguousarray(x) for x in int8)
+    rc = lib().oracle_attention_p(B, H, d, F, Hv, Wv, int(P), _p(qb), _p(kb), _p(vb), _p(prep.q8), _p(prep.k8),
+                                  _p(prep.v8t), _p(prep.s8), _p(prep.q4), _p(prep.k4), _p(prep.v4t),
+                                  _p(prep.sfq), _p(prep.sfk), _p(prep.sfv), _p(prep.g4), _p(prep.vmax),
+                                  _p(plan.cnt), _p(plan.kidx), int(flags), None if sel is None else _p(sel),
+                                  None if q8i is None else _p(q8i), None if k8i is None else _p(k8i),
+                                  None if si8 is None else _p(si8), _p(out))
+    if rc:
+        raise ValueError(f"oracle_attention_p failed ({rc})")
+    return out
+
+
+def run_prefix(q, k, v, F, Hv, Wv, P, bp8, bp4, lam=0.2, flags=7, per_row=False, bp16=0, int8=False):
+    """Whole pipeline with P prefix tokens: prepare (all blocks) -> draft and
+    assign over the video blocks -> prefix plan -> attention."""
+    prep = prepare(q, k, v, F, Hv, Wv, P)
+    Rv = F * (-(-(Hv * Wv) // BLOCK))
+    A = draft(np.ascontiguousarray(prep.desc[:, :, :, :Rv]), lam)
+    plan = prefix_plan(tiers_plan(A, bp8, bp4, per_row, bp16), -(-P // BLOCK))
+    i8 = prepare_int8(q, k, F, Hv, Wv, P) if int8 else None
+    out = attention_prefix(q, k, v, F, Hv, Wv, P, prep, plan, flags, int8=i8)
+    return prep, A, plan, out
 
 
 def attention(q, k, v, F, Hv, Wv, prep: Prepared, plan: Plan, flags: int = 7, blocks=None, int8=None) -> np.ndarray:
