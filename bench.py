@@ -154,7 +154,7 @@ def run_ours(args, w, rank, world):
     qh, kh, vh = (t.pin_memory() for t in workload_qkv(w, seed=0))
     q, k, v = (t.to(dev) for t in (qh, kh, vh))
     prep = m.alloc_prepared(dev)
-    plan = m.alloc_plan(dev)
+    plan = m.alloc_plan(dev, (w.bp8, w.bp4))
     out = torch.empty_like(q)
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
 
@@ -382,7 +382,9 @@ def main():
     t_att = r["t_attn"] * 1e-3
     achieved = (F8 + F4) / t_att / 1e12
     peak_mix = (F8 + F4) / t_roof / 1e12 if t_roof > 0 else None
-    launches_per_step = 1 + (1 + 1 + 1 + 8 + 1) + 1  # prepare; logits, softmax, select init, 8 selection passes, classify; attention
+    # prepare; logits, softmax, selection init, 8 selection passes, classify,
+    # list offsets, lists; attention
+    launches_per_step = 1 + (1 + 1 + 1 + 8 + 1 + 1 + 1) + 1
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -33,11 +33,13 @@
  *     DA2_ERR_TIMEOUT (it synchronizes the stream it is given).
  *   - Inputs are bf16, finite.  NaN / Inf inputs give undefined results.
  *
- * Geometry.  The sequence holds F frames of Hv x Wv tokens in raster order
- * (token t = f*Hv*Wv + y*Wv + x).  Each frame is split into
- * R_f = ceil(Hv*Wv/64) connected regions of balanced size (App. C.2); region
- * j of frame f is block a = f*R_f + j, R = F*R_f blocks, Npad = 64*R packed
- * slots.  Slots >= n_a of block a are padding.
+ * Geometry.  The sequence holds P prefix (text) tokens, then F frames of
+ * Hv x Wv tokens in raster order (token t = P + f*Hv*Wv + y*Wv + x).  Each
+ * frame is split into R_f = ceil(Hv*Wv/64) connected regions of balanced size
+ * (App. C.2); region j of frame f is block a = f*R_f + j (Rv = F*R_f video
+ * blocks); prefix block Rv + i holds prefix tokens 64i .. 64i+63; R = Rv +
+ * ceil(P/64) blocks, Npad = 64*R packed slots.  Slots >= n_a of block a are
+ * padding.
  */
 #ifndef DA2_H
 #define DA2_H
@@ -58,29 +60,48 @@ extern "C" {
 typedef struct {
     int B, H;      /* batch, heads */
     int d;         /* head dim: 64 or 128 */
-    int F, Hv, Wv; /* frames and latent frame size; N = F*Hv*Wv tokens */
+    int F, Hv, Wv; /* frames and latent frame size */
     int C;         /* region capacity = attention block size; must be 64 */
+    int P;         /* prefix (text) tokens before the video tokens, 0 = none;
+                      N = P + F*Hv*Wv tokens.  Prefix interactions lie outside
+                      the precision budget (App. C.1): video queries keep every
+                      prefix key and prefix queries attend to every key, on the
+                      16-bit path (which then needs the bf16 operands). */
 } da2_shape;
 
 typedef struct {
     int bp_fp8;    /* basis points of the R^2 region pairs of each head kept in FP8 */
-    int bp_fp4;    /* basis points kept in NVFP4; bp_fp8 + bp_fp4 <= 10000; the rest is skipped */
+    int bp_fp4;    /* basis points kept in NVFP4; bp_fp16 + bp_fp8 + bp_fp4 <= 10000; the rest
+                      is skipped */
     double lambda; /* max-pool branch weight of the draft map (Eq. 3); 0 = average only */
     int per_row;   /* 0: rank all R^2 pairs of a head (DraftAttention2, Sec. 3.1 and App. C.1
                       "ranks all video-region pairs within each head").  1: rank the R key
                       blocks of each query block separately, quotas floor(R bp/10^4) per row
                       (a reading of a per-query-row ranking; ties to the smaller key block). */
+    int bp_fp16;   /* basis points kept at 16 bits (bf16 operands; Table 1's 16-bit share),
+                      the highest-ranked pairs; 0 = no 16-bit tier.  Cumulative cuts:
+                      C16 = floor(n bp_fp16/10^4), C8 = floor(n (bp_fp16+bp_fp8)/10^4),
+                      Ck = floor(n (bp_fp16+bp_fp8+bp_fp4)/10^4), n = R^2 (or R per row);
+                      rank < C16 -> 16, < C8 -> 8, < Ck -> 4, else skipped (App. B.6). */
 } da2_budget;
 
 typedef struct da2_ctx* da2_handle;
 
-/* Byte sizes of every caller-owned buffer for a shape (filled by da2_sizes). */
+/* Byte sizes of every caller-owned buffer for a shape (filled by da2_sizes).
+ * R counts every block: the Rv video blocks, then the Rp = ceil(P/64) prefix
+ * blocks; the draft map, the ranking and prec cover the Rv video blocks. */
 typedef struct {
     int R, Rf, Npad;
     /* prepared operands */
     size_t desc, q8, k8, v8, q4, k4, v4, sfq, sfk, sfv, scale, vmax;
-    /* plan outputs and scratch */
-    size_t prec, cnt, kidx, A, plan_scratch;
+    /* plan outputs and scratch; kidx is the largest list size over all budgets
+       (every pair kept): da2_list_bytes gives the exact size of a budget */
+    size_t prec, cnt, off, kidx, A, plan_scratch;
+    /* optional bf16 operands of the 16-bit path */
+    size_t q16, k16, v16;
+    /* optional INT8 operands of the 8-bit phase's QK^T */
+    size_t q8i, k8i, si8;
+    int Rv, Rp;
 } da2_sizes_t;
 
 /* Prepared operands (da2_prepare output, da2_attention input).  All device.
@@ -106,25 +127,53 @@ typedef struct {
  *                               NVFP4 tile scales of Q, K, V (amax/2688).
  *   vmax  f32 [2][B][H]         per head max of the FP8 and of the NVFP4 V tile
  *                               scales (the phase units are vmax/448, vmax/2688).
+ *   q16,k16 u8 [B][H][R][128*d] optional: bf16 tiles of Q and K for the 16-bit
+ *                               path (the input values as they are), same layout
+ *                               with 2d-byte rows; slots >= n_a are zero.
+ *   v16   u8 [B][H][R][128*d]   optional: bf16 V^T (d rows x 64 slots, 128-byte
+ *                               rows), same layout.
+ *                               The three are all null (no 16-bit path) or all set.
+ *   q8i,k8i s8 [B][H][R][64*d]  optional: INT8 codes of Q and K for the 8-bit
+ *                               phase's QK^T (App. C.1: INT8 QK^T, FP8 PV), same
+ *                               layout as q8; code = RNE(x * (127/amax)) of the
+ *                               tile, clamped to +-127.
+ *   si8   f32 [2][B][H][R]      optional: their tile scales amax/127 (Q, K).
+ *                               The three are all null (FP8 QK^T) or all set;
+ *                               when set, da2_attention takes the 8-bit phase's
+ *                               scores from them.
  */
 typedef struct {
     double* desc;
     uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
     float* scale;
     float* vmax;
+    uint8_t *q16, *k16, *v16;
+    int8_t *q8i, *k8i;
+    float* si8;
 } da2_prepared;
 
 /* Plan (da2_plan output, da2_attention input).  All device.
- *   prec    u8  [B][H][R][R]  precision of pair (a,b): 8, 4 or 0 (skip)
- *   cnt     i32 [2][B][H][R]  per query block: number of FP8, of NVFP4 key blocks
- *   kidx    u16 [B][H][R][R]  row a: its FP8 key blocks ascending, then its
- *                             NVFP4 key blocks ascending (cnt entries used)
- *   A       f64 [B][H][R][R]  the draft map (Eq. 3), left readable after the call
+ *   prec    u8  [B][H][Rv][Rv] precision of video pair (a,b): 16, 8, 4 or 0 (skip)
+ *   cnt     i32 [3][B][H][R]  per query block: number of FP8, of NVFP4 and of
+ *                             16-bit key blocks (prefix blocks count as 16-bit)
+ *   off     i64 [B][H][R+1]   list offsets: query block a of head (b,h) owns
+ *                             kidx[off[b][h][a] .. off[b][h][a+1]); head (b,h)
+ *                             starts at (b*H + h) * K, K = the pairs a head keeps
+ *                             (its budgeted video pairs, plus Rv*Rp + Rp*R with
+ *                             a prefix)
+ *   kidx    u16 [B*H*K]       compact lists: row a's 16-bit key blocks ascending
+ *                             (for a video row: its 16-bit video blocks, then
+ *                             every prefix block), then its FP8 ones, then its
+ *                             NVFP4 ones (the phase order of the attention); a
+ *                             prefix row lists every block
+ *                             (da2_list_bytes bytes for the budget)
+ *   A       f64 [B][H][Rv][Rv] the draft map (Eq. 3), left readable after the call
  *   scratch                   plan_scratch bytes of working memory
  */
 typedef struct {
     uint8_t* prec;
     int32_t* cnt;
+    int64_t* off;
     uint16_t* kidx;
     double* A;
     void* scratch;
@@ -151,6 +200,13 @@ int da2_destroy(da2_handle h);
 /* Sizes of every caller-owned buffer for the handle's shape. */
 int da2_sizes(da2_handle h, da2_sizes_t* out);
 
+/* Exact byte size of the compact lists (da2_plan_bufs.kidx) under a budget:
+ * 2 bytes per kept pair, B*H*K pairs with K = floor(Rv^2 bp/10^4) (per_row =
+ * 0) or Rv*floor(Rv bp/10^4) (per_row = 1), bp = bp_fp16 + bp_fp8 + bp_fp4,
+ * plus Rv*Rp + Rp*R prefix pairs.  Errors:
+ * DA2_ERR_ARG for a null argument or a budget da2_plan would reject. */
+int da2_list_bytes(da2_handle h, const da2_budget* budget, size_t* bytes);
+
 /* Host copies of the partition tables: slot_token[Npad] (token of each packed
  * slot, -1 for padding) and n_a[R] (valid tokens per block).  Either may be
  * NULL. */
@@ -170,8 +226,9 @@ int da2_prepare(da2_handle h, const void* q, const void* k, const void* v, const
  * Tkeep = floor(R^2 (bp_fp8+bp_fp4)/10^4); ranks below T8 -> FP8, below
  * Tkeep -> NVFP4, the rest skipped; per-row lists.  With budget->per_row = 1
  * the ranking and the quotas floor(R bp/10^4) are per query block instead.
- * Errors: DA2_ERR_ARG for a budget outside [0, 10000], lambda outside [0, 1]
- * or per_row other than 0 / 1. */
+ * With bp_fp16 > 0 the three cuts of da2_budget give 16-bit, FP8 and NVFP4
+ * pairs.  Errors: DA2_ERR_ARG for a budget outside [0, 10000], lambda
+ * outside [0, 1] or per_row other than 0 / 1. */
 int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, const da2_plan_bufs* plan,
              void* stream);
 
@@ -189,8 +246,8 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
  * would stall other streams.  This entry point computes exactly what da2_plan
  * computes (same kernels, same results) but takes no scratch buffer: its
  * working memory is a fixed DA2_PLAN_STATIC_BYTES array inside the library.
- * The caller still passes the prepared operands and the four outputs (prec,
- * cnt, kidx, A, device, layouts as in da2_plan_bufs).
+ * The caller still passes the prepared operands and the five outputs (prec,
+ * cnt, off, kidx, A, device, layouts as in da2_plan_bufs).
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress); make that first call before any stream
  *     capture begins.
@@ -203,7 +260,7 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
  *     tells how much: about B*H*R*R*8 bytes plus 33 KB per head).  Other
  *     errors as da2_plan. */
 int da2_plan_static(da2_handle h, const da2_prepared* prep, const da2_budget* budget, uint8_t* prec, int32_t* cnt,
-                    uint16_t* kidx, double* A, void* stream);
+                    int64_t* off, uint16_t* kidx, double* A, void* stream);
 
 /* Block-sparse mixed-precision attention (Sec. 3.3; App. B.3, C.1).  out:
  * bf16 (device), [B][H][N][d] with strides out_strides[] in elements

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from oracle import oracle as O
-from tests.gpu_common import SMALL, gpu_run, inputs
+from tests.gpu_common import SMALL, check_compact_lists, gpu_run, inputs
 from video_dit_sparse_da2_b200.inputs import make_qkv
 
 pytestmark = pytest.mark.gpu
@@ -15,6 +15,7 @@ def _check_plan(got, A, plan):
     assert np.array_equal(got["A"].view(np.uint64), A.view(np.uint64)), "draft map differs"
     assert np.array_equal(got["prec"], plan.prec)
     assert np.array_equal(got["cnt"], plan.cnt)
+    check_compact_lists(got, plan.cnt, plan.kidx)
     B, H, R, _ = A.shape
     for b in range(B):
         for h in range(H):

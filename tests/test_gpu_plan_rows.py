@@ -37,12 +37,15 @@ def test_plan_rows_ties_by_key_block():
     _check_plan(res["plan"], A, O.assign(A, 2500, 2500, per_row=True))
 
 
-def test_plan_rows_bit_exact_wan13b():
-    B, H, d, F, Hv, Wv = 1, 12, 128, 21, 30, 52
-    res = gpu_run(B, H, d, F, Hv, Wv, 1000, 3000, per_row=True)
+@pytest.mark.parametrize("shape,bp", [((1, 12, 128, 21, 30, 52), (1000, 3000)),
+                                      ((1, 24, 128, 33, 45, 80), (500, 2500))],
+                         ids=["wan2.1-1.3b-480p", "hunyuanvideo-720p"])
+def test_plan_rows_bit_exact_full_size(shape, bp):
+    B, H, d, F, Hv, Wv = shape
+    res = gpu_run(B, H, d, F, Hv, Wv, *bp, per_row=True)
     q, k, v = inputs(B, H, d, F, Hv, Wv)
     A = O.draft(O.prepare(q, k, v, F, Hv, Wv).desc, 0.2)
-    _check_plan(res["plan"], A, O.assign(A, 1000, 3000, per_row=True))
+    _check_plan(res["plan"], A, O.assign(A, *bp, per_row=True))
 
 
 @pytest.mark.parametrize("name", ["tiny", "ragged128"])

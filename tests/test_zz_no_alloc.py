@@ -29,8 +29,9 @@ CASES = [  # (B, H, d, F, Hv, Wv, bp8, bp4, lam): the second needs ~27 MB of wor
 ]
 
 
-def _plan_bytes(plan, B, H, R):
+def _plan_bytes(plan, B, H, R, list_bytes):
     g = layouts.plan_to_logical(plan.bufs, B, H, R)
+    g["kidx_flat"] = g["kidx_flat"][: list_bytes // 2]
     return {k: np.ascontiguousarray(v).view(np.uint8).copy() for k, v in g.items()}
 
 
@@ -43,23 +44,24 @@ def test_plan_static_matches_plan_twice(case, per_row):
     q, k, v = (t.cuda() for t in make_qkv(B, H, F * Hv * Wv, d, seed=11))
     prep = m.alloc_prepared()
     m.prepare(q, k, v, prep)
-    ref = m.alloc_plan()
+    nlist = m.list_bytes(bp8, bp4, per_row)
+    ref = m.alloc_plan(budget=(bp8, bp4, per_row))
     m.plan(prep, ref, bp8, bp4, lam, per_row=per_row)
     torch.cuda.synchronize()
-    want = _plan_bytes(ref, B, H, m.R)
+    want = _plan_bytes(ref, B, H, m.R, nlist)
     for call in range(2):
-        got_plan = m.alloc_plan()
+        got_plan = m.alloc_plan(budget=(bp8, bp4, per_row))
         for t in got_plan.bufs.values():
             t.fill_(0xA5)  # outputs start as garbage: everything must be written
         m.plan_static(prep, got_plan, bp8, bp4, lam, per_row=per_row)
         torch.cuda.synchronize()
         m.check_status()
-        got = _plan_bytes(got_plan, B, H, m.R)
+        got = _plan_bytes(got_plan, B, H, m.R, nlist)
         R = m.R
         cnt = want["cnt"].view(np.int32).reshape(2, B, H, R)
         n = (cnt[0] + cnt[1])[..., None]
         listed = np.arange(R)[None, None, None, :] < n
-        for key in ("A", "prec", "cnt"):
+        for key in ("A", "prec", "cnt", "off", "kidx_flat"):
             assert np.array_equal(got[key], want[key]), (call, key)
         gk = got["kidx"].view(np.uint16).reshape(B, H, R, R)
         wk = want["kidx"].view(np.uint16).reshape(B, H, R, R)
@@ -74,7 +76,7 @@ def test_plan_static_refuses_large_shapes():
     p = small.data_ptr()
     ptrs = da2.PreparedPtrs(*([p] * 12))
     b = da2.Budget(1000, 1000, 0.2)
-    rc = da2.lib().da2_plan_static(m.handle, ctypes.byref(ptrs), ctypes.byref(b), p, p, p, p, None)
+    rc = da2.lib().da2_plan_static(m.handle, ctypes.byref(ptrs), ctypes.byref(b), p, p, p, p, p, None)
     assert rc == da2.ERR_ARG
     torch.cuda.synchronize()
     assert not small.any()  # nothing was enqueued

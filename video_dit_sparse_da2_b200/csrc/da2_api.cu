@@ -13,7 +13,8 @@
 
 struct da2_ctx {
     da2_shape shape{};
-    int Rf = 0, R = 0, N = 0, Npad = 0;
+    int Rf = 0, R = 0, N = 0, Npad = 0;  // R: all blocks (video, then prefix)
+    int Rv = 0, Rp = 0;                    // video blocks, prefix blocks
     int device = 0, num_sms = 0;
     std::vector<int32_t> slot_token, n_a;  // host copies
     int32_t* d_slot_token = nullptr;       // [Npad]
@@ -39,12 +40,24 @@ bool prepared_ok(const da2_prepared* p) {
     const void* ptrs[] = {p->desc, p->q8, p->k8, p->v8, p->q4, p->k4, p->v4, p->sfq, p->sfk, p->sfv, p->scale, p->vmax};
     for (const void* q : ptrs)
         if (!q || !aligned16(q)) return false;
+    // the 16-bit operands: all three or none
+    const bool any16 = p->q16 || p->k16 || p->v16, all16 = p->q16 && p->k16 && p->v16;
+    if (any16 && (!all16 || !aligned16(p->q16) || !aligned16(p->k16) || !aligned16(p->v16))) return false;
+    // the INT8 QK^T operands: all three or none
+    const bool anyi = p->q8i || p->k8i || p->si8, alli = p->q8i && p->k8i && p->si8;
+    if (anyi && (!alli || !aligned16(p->q8i) || !aligned16(p->k8i) || !aligned16(p->si8))) return false;
     return true;
+}
+
+bool budget_ok(const da2_budget* b) {
+    return b && b->bp_fp8 >= 0 && b->bp_fp4 >= 0 && b->bp_fp16 >= 0 &&
+           (long long)b->bp_fp16 + b->bp_fp8 + b->bp_fp4 <= 10000 && b->lambda >= 0.0 && b->lambda <= 1.0 &&
+           (b->per_row == 0 || b->per_row == 1);
 }
 
 bool plan_ok(const da2_plan_bufs* p) {
     if (!p) return false;
-    const void* ptrs[] = {p->prec, p->cnt, p->kidx, p->A, p->scratch};
+    const void* ptrs[] = {p->prec, p->cnt, p->off, p->kidx, p->A, p->scratch};
     for (const void* q : ptrs)
         if (!q || !aligned16(q)) return false;
     return true;
@@ -78,8 +91,9 @@ int da2_create(const da2_shape* s, da2_handle* out) {
     if (s->B <= 0 || s->H <= 0 || s->F <= 0 || s->Hv <= 0 || s->Wv <= 0) return DA2_ERR_ARG;
     if (s->d != 64 && s->d != 128) return DA2_ERR_ARG;
     if (s->C != 64) return DA2_ERR_ARG;
+    if (s->P < 0 || s->P > (1 << 20)) return DA2_ERR_ARG;
     const long long n = (long long)s->Hv * s->Wv;
-    const long long Rf = (n + 63) / 64, R = Rf * s->F;
+    const long long Rf = (n + 63) / 64, R = Rf * s->F + (s->P + 63) / 64;
     if (R > 4096 || (long long)s->B * s->H * R * R > (1ll << 40)) return DA2_ERR_ARG;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -94,19 +108,28 @@ int da2_create(const da2_shape* s, da2_handle* out) {
     if (!h) return DA2_ERR_CUDA;
     h->shape = *s;
     h->Rf = part.Rf;
-    h->R = s->F * part.Rf;
-    h->N = s->F * (int)n;
+    h->Rv = s->F * part.Rf;
+    h->Rp = (s->P + 63) / 64;
+    h->R = h->Rv + h->Rp;
+    h->N = s->P + s->F * (int)n;
     h->Npad = 64 * h->R;
     h->device = dev;
     h->num_sms = prop.multiProcessorCount;
     h->slot_token.assign(h->Npad, -1);
     h->n_a.assign(h->R, 0);
+    // video tokens follow the P prefix tokens; the prefix blocks (64
+    // consecutive prefix tokens each) follow the video blocks
     for (int f = 0; f < s->F; ++f) {
         for (int j = 0; j < part.Rf; ++j) h->n_a[f * part.Rf + j] = part.size[j];
         for (long long c = 0; c < n; ++c) {
             const int a = f * part.Rf + part.region[c];
-            h->slot_token[(size_t)a * 64 + part.slot[c]] = (int32_t)(f * n + c);
+            h->slot_token[(size_t)a * 64 + part.slot[c]] = (int32_t)(s->P + f * n + c);
         }
+    }
+    for (int i = 0; i < h->Rp; ++i) {
+        const int a = h->Rv + i, cnt = s->P - 64 * i < 64 ? s->P - 64 * i : 64;
+        h->n_a[a] = cnt;
+        for (int j = 0; j < cnt; ++j) h->slot_token[(size_t)a * 64 + j] = 64 * i + j;
     }
     if ((e = cudaMalloc(&h->d_slot_token, sizeof(int32_t) * h->Npad)) != cudaSuccess ||
         (e = cudaMalloc(&h->d_n_a, sizeof(int32_t) * h->R)) != cudaSuccess ||
@@ -152,11 +175,13 @@ int da2_destroy(da2_handle h) {
 
 int da2_sizes(da2_handle h, da2_sizes_t* o) {
     if (!h || !o) return DA2_ERR_ARG;
-    const size_t BH = (size_t)h->shape.B * h->shape.H, R = h->R, d = h->shape.d;
+    const size_t BH = (size_t)h->shape.B * h->shape.H, R = h->R, Rv = h->Rv, d = h->shape.d;
     std::memset(o, 0, sizeof(*o));
     o->R = h->R;
     o->Rf = h->Rf;
     o->Npad = h->Npad;
+    o->Rv = h->Rv;
+    o->Rp = h->Rp;
     o->desc = 4 * BH * R * d * sizeof(double);
     o->q8 = o->k8 = o->v8 = BH * R * 64 * d;
     o->q4 = o->k4 = o->v4 = BH * R * 32 * d;
@@ -164,11 +189,25 @@ int da2_sizes(da2_handle h, da2_sizes_t* o) {
     o->sfk = o->sfv = BH * R * 512;
     o->scale = 6 * BH * R * sizeof(float);
     o->vmax = 2 * BH * sizeof(float);
-    o->prec = BH * R * R;
-    o->cnt = 2 * BH * R * sizeof(int32_t);
+    o->prec = BH * Rv * Rv;
+    o->cnt = 3 * BH * R * sizeof(int32_t);
+    o->off = BH * (R + 1) * sizeof(int64_t);
     o->kidx = BH * R * R * sizeof(uint16_t);
-    o->A = BH * R * R * sizeof(double);
-    o->plan_scratch = da2::plan_scratch_bytes((int)BH, (int)R);
+    o->A = BH * Rv * Rv * sizeof(double);
+    o->plan_scratch = da2::plan_scratch_bytes((int)BH, (int)Rv);
+    o->q16 = o->k16 = o->v16 = BH * R * 128 * d;
+    o->q8i = o->k8i = BH * R * 64 * d;
+    o->si8 = 2 * BH * R * sizeof(float);
+    return DA2_OK;
+}
+
+int da2_list_bytes(da2_handle h, const da2_budget* budget, size_t* bytes) {
+    if (!h || !bytes || !budget_ok(budget)) return DA2_ERR_ARG;
+    const size_t BH = (size_t)h->shape.B * h->shape.H;
+    *bytes = BH *
+             (size_t)da2::plan_kept_per_head(h->Rv, h->Rp, budget->bp_fp16, budget->bp_fp8, budget->bp_fp4,
+                                             budget->per_row) *
+             sizeof(uint16_t);
     return DA2_OK;
 }
 
@@ -190,6 +229,7 @@ int da2_prepare(da2_handle h, const void* q, const void* k, const void* v, const
     a.H = h->shape.H;
     a.d = h->shape.d;
     a.R = h->R;
+    a.Rv = h->Rv;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.k = static_cast<const __nv_bfloat16*>(k);
     a.v = static_cast<const __nv_bfloat16*>(v);
@@ -202,22 +242,27 @@ int da2_prepare(da2_handle h, const void* q, const void* k, const void* v, const
     a.q8 = out->q8; a.k8 = out->k8; a.v8 = out->v8;
     a.q4 = out->q4; a.k4 = out->k4; a.v4 = out->v4;
     a.sfq = out->sfq; a.sfk = out->sfk; a.sfv = out->sfv;
+    a.q16 = out->q16; a.k16 = out->k16; a.v16 = out->v16;
+    a.q8i = out->q8i; a.k8i = out->k8i; a.si8 = out->si8;
     a.scale = out->scale;
     a.vmax = out->vmax;
+    a.status = h->d_status;
+    a.wait_ns = h->wait_ns;
+    a.num_sms = h->num_sms;
     cudaError_t e = da2::launch_prepare(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DA2_OK : cuda_fail(e);
 }
 
 int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, const da2_plan_bufs* plan,
              void* stream) {
-    if (!h || !prepared_ok(prep) || !budget || !plan_ok(plan)) return DA2_ERR_ARG;
-    if (budget->bp_fp8 < 0 || budget->bp_fp4 < 0 || budget->bp_fp8 + budget->bp_fp4 > 10000) return DA2_ERR_ARG;
-    if (!(budget->lambda >= 0.0 && budget->lambda <= 1.0)) return DA2_ERR_ARG;
-    if (budget->per_row != 0 && budget->per_row != 1) return DA2_ERR_ARG;
+    if (!h || !prepared_ok(prep) || !budget_ok(budget) || !plan_ok(plan)) return DA2_ERR_ARG;
     da2::PlanArgs a{};
     a.BH = h->shape.B * h->shape.H;
-    a.R = h->R;
+    a.R = h->Rv;   // the ranking covers the video blocks
+    a.Rt = h->R;   // lists, counts and prepared operands cover every block
+    a.Rp = h->Rp;
     a.d = h->shape.d;
+    a.bp16 = budget->bp_fp16;
     a.bp8 = budget->bp_fp8;
     a.bp4 = budget->bp_fp4;
     a.lambda = budget->lambda;
@@ -226,6 +271,7 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
     a.A = plan->A;
     a.prec = plan->prec;
     a.cnt = plan->cnt;
+    a.off = reinterpret_cast<long long*>(plan->off);
     a.kidx = plan->kidx;
     a.status = h->d_status;
     a.num_sms = h->num_sms;
@@ -251,9 +297,12 @@ int da2_attention(da2_handle h, const da2_prepared* prep, const da2_plan_bufs* p
     a.q8 = prep->q8; a.k8 = prep->k8; a.v8 = prep->v8;
     a.q4 = prep->q4; a.k4 = prep->k4; a.v4 = prep->v4;
     a.sfq = prep->sfq; a.sfk = prep->sfk; a.sfv = prep->sfv;
+    a.q16 = prep->q16; a.k16 = prep->k16; a.v16 = prep->v16;
+    a.q8i = prep->q8i; a.k8i = prep->k8i; a.si8 = prep->si8;
     a.scale = prep->scale;
     a.vmax = prep->vmax;
     a.cnt = plan->cnt;
+    a.off = reinterpret_cast<const long long*>(plan->off);
     a.kidx = plan->kidx;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.o0 = out_strides[0];

@@ -9,15 +9,22 @@ struct da2_ctx;
 namespace da2 {
 
 struct PrepareArgs {
-    int B, H, d, R;
+    int B, H, d, R;            // R: every block (video, then prefix)
+    int Rv;                    // video blocks (the V maxima cover these)
     const __nv_bfloat16 *q, *k, *v;
     long long s0, s1, s2;      // element strides of batch, head, token
     const int32_t* slot_token; // [64 R] token of each slot, -1 = padding
     const int32_t* n_a;        // [R]
     double* desc;
     uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
+    uint8_t *q16, *k16, *v16;    // bf16 tiles of the 16-bit path, or all null
+    int8_t *q8i, *k8i;           // INT8 tiles of Q and K, or null
+    float* si8;                  // [2][BH][R] their tile scales, or null
     float* scale;
     float* vmax;
+    unsigned* status;            // handle status word (bounded waits)
+    unsigned long long wait_ns;  // limit of every bounded device-side wait
+    int num_sms;
 };
 cudaError_t launch_prepare(const PrepareArgs& p, cudaStream_t stream);
 
@@ -38,24 +45,28 @@ struct __align__(16) SelectTarget {
 };
 
 struct PlanArgs {
-    int BH, R, d;
-    int bp8, bp4;
+    int BH, R, d;            // R: video blocks (draft map, ranking, prec, A)
+    int Rt, Rp;              // every block (Rv + Rp prefix blocks): descriptors, counts, lists
+    int bp16, bp8, bp4;
     double lambda;
     int per_row;             // 1: quotas and ranking per query block instead of per head
     const double* desc;      // [4][BH][R][d]
     double* A;               // [BH][R][R] (first holds the average-branch logits)
     double* Lmax;            // [BH][R][R] max-branch logits (scratch)
     unsigned long long* abits_minmax;  // [BH][2] (scratch)
-    SelectTarget* sel;       // [BH][2] (scratch)
-    unsigned int* hist;      // [BH][2][4096] (scratch)
+    SelectTarget* sel;       // [BH][3] (scratch): 16-bit, 8-bit, kept cuts
+    unsigned int* hist;      // [BH][3][4096] (scratch)
     unsigned int* done_count;  // [BH] finished histogram CTAs of the current pass (scratch)
     uint8_t* prec;           // [BH][R][R]
-    int32_t* cnt;            // [2][BH][R]
-    uint16_t* kidx;          // [BH][R][R]
+    int32_t* cnt;            // [3][BH][R]: 8-bit, 4-bit, 16-bit counts
+    long long* off;          // [BH][R+1] list offsets (positions in kidx)
+    uint16_t* kidx;          // [BH * kept per head] compact lists
     unsigned* status;
     int num_sms;             // multiprocessors of the device (grid sizing)
 };
 size_t plan_scratch_bytes(int BH, int R);
+// Kept pairs of one head under a budget (the length of its part of kidx).
+long long plan_kept_per_head(int Rv, int Rp, int bp16, int bp8, int bp4, int per_row);
 void plan_carve_scratch(PlanArgs* p, void* scratch);
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream);
 
@@ -64,10 +75,14 @@ struct AttnArgs {
     const int32_t* slot_token;  // [64 R]
     const int32_t* n_a;         // [R]
     const uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
+    const uint8_t *q16, *k16, *v16;  // bf16 tiles of the 16-bit path, or all null
+    const int8_t *q8i, *k8i;         // INT8 Q/K tiles: the 8-bit phase's QK^T in INT8, or null
+    const float* si8;                // [2][BH][R] their tile scales
     const float* scale;  // [6][BH][R]
     const float* vmax;   // [2][BH]
-    const int32_t* cnt;  // [2][BH][R]
-    const uint16_t* kidx;  // [BH][R][R]
+    const int32_t* cnt;  // [3][BH][R]: 8-bit, 4-bit, 16-bit counts
+    const long long* off;  // [BH][R+1]
+    const uint16_t* kidx;  // compact lists at off
     __nv_bfloat16* out;
     long long o0, o1, o2;  // element strides of the output
     unsigned* status;

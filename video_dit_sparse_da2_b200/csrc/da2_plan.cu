@@ -12,9 +12,11 @@
 // exp_fixed is a Cody-Waite reduction with a two-part ln2 and a degree-13
 // Taylor polynomial in Horner form (fma), scaled by 2^k; results below the
 // normal range are flushed to zero.  The ranking is an exact radix selection
-// of the T8-th and Tkeep-th largest 96-bit keys (A bits : ~pair index), i.e.
+// of the C16-th, C8-th and Ck-th largest 96-bit keys (A bits : ~pair index)
+// -- the cumulative cuts of the 16-bit, 8-bit and kept tiers --, i.e.
 // A descending with ties to the smaller pair index a*R+b, followed by an
-// exact classification and an ordered per-row compaction of the lists.
+// exact classification, a scan of the rows' counts into list offsets and an
+// ordered compaction of every row's list at its offset.
 #include <algorithm>
 #include <cfloat>
 
@@ -66,9 +68,11 @@ __global__ void __launch_bounds__(kLgThreads, 1) logits_kernel(PlanArgs p, doubl
     const int R = p.R, bh = blockIdx.z >> 1, branch = blockIdx.z & 1;
     const int a0 = blockIdx.y * kLgTile, b0 = blockIdx.x * kLgTile;
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-    const size_t plane = (size_t)p.BH * R * D;
-    const double* Qs = p.desc + (size_t)branch * plane + (size_t)bh * R * D;
-    const double* Ks = p.desc + (size_t)(2 + branch) * plane + (size_t)bh * R * D;
+    // descriptors of every block are stored (Rt per head); the draft uses the
+    // R video blocks
+    const size_t plane = (size_t)p.BH * p.Rt * D;
+    const double* Qs = p.desc + (size_t)branch * plane + (size_t)bh * p.Rt * D;
+    const double* Ks = p.desc + (size_t)(2 + branch) * plane + (size_t)bh * p.Rt * D;
 
     // staging: thread t moves channel pairs of rows (t + 256 it) % 128
     double2 rq[4], rk[4];
@@ -243,6 +247,8 @@ struct Key {
     unsigned int lo;
 };
 
+constexpr int kTargets = 3;  // selection targets per head (16-bit, 8-bit, kept cuts)
+
 __device__ __forceinline__ void top_mask(int nbits, unsigned long long* mh, unsigned int* ml) {
     *mh = nbits <= 0 ? 0ull : (nbits >= 64 ? ~0ull : (~0ull << (64 - nbits)));
     const int nl = nbits - 64;
@@ -257,17 +263,19 @@ __device__ __forceinline__ unsigned digit_at(Key k, int pos, int w) {
     return (unsigned)((k.hi << (32 - pos)) | (unsigned long long)(k.lo >> pos)) & mask;
 }
 
-__global__ void select_init_kernel(PlanArgs p, long long T8, long long Tk) {
+// Targets of a head, in order: the C16-th, C8-th and Ck-th largest keys (the
+// cumulative cuts of the 16-bit, 8-bit and kept tiers); a cut of 0 is "none".
+__global__ void select_init_kernel(PlanArgs p, long long C16, long long C8, long long Ck) {
     const int bh = blockIdx.x * blockDim.x + threadIdx.x;
     if (bh >= p.BH) return;
     const unsigned long long lo = p.abits_minmax[bh], hi = p.abits_minmax[p.BH + bh];
     const int c = (lo == hi) ? 64 : __clzll((long long)(lo ^ hi));
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < kTargets; ++t) {
         SelectTarget s;
         s.nbits = c;
         s.p_hi = (c >= 64) ? lo : (c == 0 ? 0ull : (lo & (~0ull << (64 - c))));
         s.p_lo = 0u;
-        s.need = t == 0 ? T8 : Tk;
+        s.need = t == 0 ? C16 : (t == 1 ? C8 : Ck);
         s.unique = 0;
         s.found = 0;
         s.matches = (long long)p.R * p.R;
@@ -275,7 +283,7 @@ __global__ void select_init_kernel(PlanArgs p, long long T8, long long Tk) {
         s.done = s.none;
         s.key_hi = 0ull;
         s.key_lo = 0u;
-        p.sel[bh * 2 + t] = s;
+        p.sel[bh * kTargets + t] = s;
     }
 }
 
@@ -286,8 +294,8 @@ constexpr long long kHistDirect = 1ll << 14;     // at most this many matching k
 // Choose the digit that holds the sought rank of target t of head bh (one
 // warp), from the completed histogram of the pass, and clear the histogram.
 __device__ void select_scan_warp(PlanArgs& p, int bh, int t, int lane) {
-    unsigned* gh = p.hist + ((size_t)bh * 2 + t) * 4096;
-    SelectTarget* sp = &p.sel[bh * 2 + t];
+    unsigned* gh = p.hist + ((size_t)bh * kTargets + t) * 4096;
+    SelectTarget* sp = &p.sel[bh * kTargets + t];
     // from L2: another CTA of this pass may have recorded the unique key
     SelectTarget s;
     static_assert(sizeof(SelectTarget) % 16 == 0, "SelectTarget is read as 16-byte words");
@@ -350,27 +358,40 @@ __device__ void select_scan_warp(PlanArgs& p, int bh, int t, int lane) {
 // the digits (select_scan_warp).  A target whose prefix matches one key
 // records that key here and is marked done by that pass's scan, so the
 // `done` flags do not change while a pass runs.
+template <int NT>
 __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, int chunk) {
-    __shared__ unsigned h[2][4096];
+    extern __shared__ unsigned h_dyn[];  // [NT][4096]
     __shared__ int is_last;
+    constexpr int t0 = kTargets - NT;     // with no 16-bit tier only the last two targets are live
     const int bh = blockIdx.y, tid = threadIdx.x;
-    SelectTarget s[2] = {p.sel[bh * 2], p.sel[bh * 2 + 1]};
-    if (s[0].done && s[1].done) return;
-    bool in_smem[2];
-    for (int t = 0; t < 2; ++t) in_smem[t] = !s[t].done && !s[t].unique && s[t].matches > kHistDirect;
-    if (in_smem[0] || in_smem[1]) {
-        for (int i = tid; i < 2 * 4096; i += kHistThreads) (&h[0][0])[i] = 0u;
+    SelectTarget s[NT];
+    bool all_done = true;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        s[t] = p.sel[bh * kTargets + t0 + t];
+        all_done = all_done && s[t].done;
+    }
+    if (all_done) return;
+    bool in_smem[NT], any_smem = false;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        in_smem[t] = !s[t].done && !s[t].unique && s[t].matches > kHistDirect;
+        any_smem = any_smem || in_smem[t];
+    }
+    if (any_smem) {
+        for (int i = tid; i < NT * 4096; i += kHistThreads) h_dyn[i] = 0u;
         __syncthreads();
     }
-    unsigned long long mh[2];
-    unsigned ml[2];
-    int w[2], pos[2];
-    for (int t = 0; t < 2; ++t) {
+    unsigned long long mh[NT];
+    unsigned ml[NT];
+    int w[NT], pos[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
         top_mask(s[t].nbits, &mh[t], &ml[t]);
         w[t] = min(12, 96 - s[t].nbits);
         pos[t] = 96 - s[t].nbits - w[t];
     }
-    unsigned* gh = p.hist + (size_t)bh * 2 * 4096;
+    unsigned* gh = p.hist + ((size_t)bh * kTargets + t0) * 4096;
     const size_t RR = (size_t)p.R * p.R;
     const size_t begin = (size_t)blockIdx.x * chunk;
     const double* Ah = p.A + (size_t)bh * RR;
@@ -379,15 +400,15 @@ __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, i
         k.hi = (unsigned long long)__double_as_longlong(a);
         k.lo = 0xFFFFFFFFu - (unsigned)i;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < NT; ++t) {
             if (s[t].done) continue;
             if (((k.hi ^ s[t].p_hi) & mh[t]) || ((k.lo ^ s[t].p_lo) & ml[t])) continue;
             if (s[t].unique) {
-                p.sel[bh * 2 + t].key_hi = k.hi;
-                p.sel[bh * 2 + t].key_lo = k.lo;
-                p.sel[bh * 2 + t].found = 1;
+                p.sel[bh * kTargets + t0 + t].key_hi = k.hi;
+                p.sel[bh * kTargets + t0 + t].key_lo = k.lo;
+                p.sel[bh * kTargets + t0 + t].found = 1;
             } else if (in_smem[t]) {
-                atomicAdd(&h[t][digit_at(k, pos[t], w[t])], 1u);
+                atomicAdd(&h_dyn[t * 4096 + digit_at(k, pos[t], w[t])], 1u);
             } else {
                 atomicAdd(&gh[t * 4096 + digit_at(k, pos[t], w[t])], 1u);
             }
@@ -407,10 +428,10 @@ __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, i
         for (int u = 0; u < 4; ++u)
             if (idx[u] < RR) count(idx[u], a[u]);
     }
-    if (in_smem[0] || in_smem[1]) {
+    if (any_smem) {
         __syncthreads();
-        for (int i = tid; i < 2 * 4096; i += kHistThreads) {
-            const unsigned v = (&h[0][0])[i];
+        for (int i = tid; i < NT * 4096; i += kHistThreads) {
+            const unsigned v = h_dyn[i];
             if (v) atomicAdd(&gh[i], v);
         }
     }
@@ -421,74 +442,143 @@ __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, i
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    if (tid < 64) select_scan_warp(p, bh, tid >> 5, tid & 31);
+    if (tid < 32 * NT) select_scan_warp(p, bh, t0 + (tid >> 5), tid & 31);
     if (tid == 0) p.done_count[bh] = 0u;
 }
 
 // ---------------------------------------------------------------- classify
-// One warp per (head, query region): precision of every pair, then the
-// ordered list of 8-bit key blocks followed by the 4-bit key blocks.
+// One warp per (head, query region): precision of every pair (16, 8, 4 or 0)
+// and the row's numbers of 8-bit, 4-bit and 16-bit key blocks.
 __global__ void __launch_bounds__(128) classify_kernel(PlanArgs p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t row = (size_t)blockIdx.x * 4 + warp;
     const int R = p.R;
     if (row >= (size_t)p.BH * R) return;
     const int bh = (int)(row / R), a = (int)(row % R);
-    const SelectTarget s8 = p.sel[bh * 2], sk = p.sel[bh * 2 + 1];
+    const SelectTarget s16 = p.sel[bh * kTargets], s8 = p.sel[bh * kTargets + 1], sk = p.sel[bh * kTargets + 2];
     const double* Arow = p.A + row * R;
     uint8_t* prow = p.prec + row * R;
-    uint16_t* krow = p.kidx + row * R;
-    const unsigned lt = (1u << lane) - 1u;
     auto ge = [](Key k, const SelectTarget& s) {
         return !s.none && (k.hi > s.key_hi || (k.hi == s.key_hi && k.lo >= s.key_lo));
     };
-    int n8 = 0;
+    int n16 = 0, n8 = 0, n4 = 0;
     for (int b0 = 0; b0 < R; b0 += 32) {
         const int b = b0 + lane;
-        bool is8 = false;
+        bool is16 = false, is8 = false, is4 = false;
         if (b < R) {
             Key k;
             k.hi = (unsigned long long)__double_as_longlong(Arow[b]);
             k.lo = 0xFFFFFFFFu - (unsigned)(a * R + b);
-            is8 = ge(k, s8);
-            const bool keep = ge(k, sk);
-            prow[b] = is8 ? 8 : (keep ? 4 : 0);
+            is16 = ge(k, s16);
+            is8 = !is16 && ge(k, s8);
+            is4 = !is16 && !is8 && ge(k, sk);
+            prow[b] = is16 ? 16 : (is8 ? 8 : (is4 ? 4 : 0));
         }
-        const unsigned m = __ballot_sync(0xffffffffu, is8);
-        if (is8) krow[n8 + __popc(m & lt)] = (uint16_t)b;
-        n8 += __popc(m);
-    }
-    __syncwarp();
-    int n4 = 0;
-    for (int b0 = 0; b0 < R; b0 += 32) {
-        const int b = b0 + lane;
-        const bool is4 = b < R && prow[b] == 4;
-        const unsigned m = __ballot_sync(0xffffffffu, is4);
-        if (is4) krow[n8 + n4 + __popc(m & lt)] = (uint16_t)b;
-        n4 += __popc(m);
+        n16 += __popc(__ballot_sync(0xffffffffu, is16));
+        n8 += __popc(__ballot_sync(0xffffffffu, is8));
+        n4 += __popc(__ballot_sync(0xffffffffu, is4));
     }
     if (lane == 0) {
-        p.cnt[row] = n8;
-        p.cnt[(size_t)p.BH * R + row] = n4;
+        const size_t BHRt = (size_t)p.BH * p.Rt, rt = (size_t)bh * p.Rt + a;
+        p.cnt[rt] = n8;
+        p.cnt[BHRt + rt] = n4;
+        p.cnt[2 * BHRt + rt] = n16 + p.Rp;  // every prefix key is kept at 16 bits
+    }
+}
+
+// ---------------------------------------------------------------- lists
+// Compact lists: row a of head bh owns kidx[off[bh][a] .. off[bh][a+1]).
+// The kept pairs of a head number exactly `per_head` (the quota), so head bh
+// starts at bh * per_head; one warp per head scans its rows' counts.
+__global__ void offsets_kernel(PlanArgs p, long long per_head) {
+    const int bh = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (bh >= p.BH) return;
+    const int Rt = p.Rt;
+    const size_t BHRt = (size_t)p.BH * Rt;
+    long long base = (long long)bh * per_head;
+    long long* off = p.off + (size_t)bh * (Rt + 1);
+    for (int a0 = 0; a0 < Rt; a0 += 32) {
+        const int a = a0 + lane;
+        const size_t row = (size_t)bh * Rt + a;
+        // a prefix row keeps every block at 16 bits (non-sparse, App. C.1)
+        const long long n = a >= Rt ? 0 : (a >= p.R ? (long long)Rt
+                                                     : (long long)p.cnt[row] + p.cnt[BHRt + row] + p.cnt[2 * BHRt + row]);
+        long long incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (a < Rt) {
+            off[a] = base + incl - n;
+            if (a >= p.R) {
+                p.cnt[row] = 0;
+                p.cnt[BHRt + row] = 0;
+                p.cnt[2 * BHRt + row] = Rt;
+            }
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+        off[Rt] = base;
+        if (base != (long long)(bh + 1) * per_head) atomicOr(p.status, DA2_DEV_BADINDEX);
+    }
+}
+
+// One warp per (head, query region): the row's 16-bit key blocks ascending,
+// then its 8-bit ones, then its 4-bit ones, at the row's offset.
+__global__ void __launch_bounds__(128) lists_kernel(PlanArgs p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t row = (size_t)blockIdx.x * 4 + warp;
+    const int R = p.R, Rt = p.Rt;
+    if (row >= (size_t)p.BH * Rt) return;
+    const int bh = (int)(row / Rt), a = (int)(row % Rt);
+    uint16_t* krow = p.kidx + p.off[(size_t)bh * (Rt + 1) + a];
+    if (a >= R) {
+        // prefix row: every block, ascending (non-sparse, App. C.1)
+        for (int b = lane; b < Rt; b += 32) krow[b] = (uint16_t)b;
+        return;
+    }
+    const uint8_t* prow = p.prec + ((size_t)bh * R + a) * R;
+    const unsigned lt = (1u << lane) - 1u;
+    const size_t BHRt = (size_t)p.BH * Rt;
+    // 16-bit: the video blocks of the budget, then every prefix block
+    const int n16 = p.cnt[2 * BHRt + row] - p.Rp, n8 = p.cnt[row];
+    for (int i = lane; i < p.Rp; i += 32) krow[n16 + i] = (uint16_t)(R + i);
+    int i16 = 0, i8 = 0, i4 = 0;
+    for (int b0 = 0; b0 < R; b0 += 32) {
+        const int b = b0 + lane;
+        const int pr = b < R ? prow[b] : 0;
+        const unsigned m16 = __ballot_sync(0xffffffffu, pr == 16);
+        const unsigned m8 = __ballot_sync(0xffffffffu, pr == 8);
+        const unsigned m4 = __ballot_sync(0xffffffffu, pr == 4);
+        if (pr == 16) krow[i16 + __popc(m16 & lt)] = (uint16_t)b;
+        if (pr == 8) krow[n16 + p.Rp + i8 + __popc(m8 & lt)] = (uint16_t)b;
+        if (pr == 4) krow[n16 + p.Rp + n8 + i4 + __popc(m4 & lt)] = (uint16_t)b;
+        i16 += __popc(m16);
+        i8 += __popc(m8);
+        i4 += __popc(m4);
     }
 }
 
 // ---------------------------------------------------------------- per-row ranking
 // Ranking option per query block (a reading of a per-query-row ranking; the
-// pages rank all R^2 pairs of a head).  One CTA per row finds the T8-th and
-// Tkeep-th largest 76-bit keys K = (A bits : 0xFFF - b) -- A descending, ties
-// to the smaller key block b (A >= 0, so its bits order as the values) -- by
-// a radix selection over 8-bit digits in shared memory, then gives each key
-// block 8 (K >= K_T8), 4 (K >= K_Tkeep) or 0 and writes the row's lists as the
-// classification does.
+// pages rank all R^2 pairs of a head).  One CTA per row finds the C16-th,
+// C8-th and Ck-th largest 76-bit keys K = (A bits : 0xFFF - b) -- A
+// descending, ties to the smaller key block b (A >= 0, so its bits order as
+// the values) -- by a radix selection over 8-bit digits in shared memory,
+// then gives each key block 16 (K >= K_C16), 8 (K >= K_C8), 4 (K >= K_Ck) or
+// 0 and counts the row's blocks per precision as the classification does.
 constexpr int kRowRankThreads = 256;
 typedef unsigned __int128 u128;
 
-__global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, long long T8, long long Tk) {
-    __shared__ unsigned hist[2][256];
-    __shared__ u128 pre[2];      // selected prefix (digits in place)
-    __shared__ int nbits[2];     // bits of the prefix already fixed
-    __shared__ long long need[2];  // rank still sought inside the prefix (1-based)
+__global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, long long C16, long long C8,
+                                                                   long long Ck) {
+    constexpr int NT = kTargets;
+    __shared__ unsigned hist[NT][256];
+    __shared__ u128 pre[NT];        // selected prefix (digits in place)
+    __shared__ int nbits[NT];       // bits of the prefix already fixed
+    __shared__ long long need[NT];  // rank still sought inside the prefix (1-based)
     __shared__ uint8_t prec_s[4096];
     const int R = p.R, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t row = blockIdx.x;
@@ -496,27 +586,28 @@ __global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, l
     auto keyof = [&](int b) -> u128 {
         return ((u128)(unsigned long long)__double_as_longlong(Arow[b]) << 12) | (u128)(0xFFFu - (unsigned)b);
     };
-    if (tid < 2) {
+    if (tid < NT) {
         pre[tid] = 0;
         nbits[tid] = 0;
-        need[tid] = tid == 0 ? T8 : Tk;
+        need[tid] = tid == 0 ? C16 : (tid == 1 ? C8 : Ck);
     }
     __syncthreads();
     for (int pass = 0; pass < 10; ++pass) {  // 76 bits in 8-bit digits (the last one 4 bits)
-        for (int i = tid; i < 2 * 256; i += kRowRankThreads) (&hist[0][0])[i] = 0u;
+        for (int i = tid; i < NT * 256; i += kRowRankThreads) (&hist[0][0])[i] = 0u;
         __syncthreads();
-        int w[2], pos[2];
-        bool live[2];
-        for (int t = 0; t < 2; ++t) {
+        int w[NT], pos[NT];
+        bool live[NT], any_live = false;
+        for (int t = 0; t < NT; ++t) {
             live[t] = need[t] > 0 && nbits[t] < 76;
             w[t] = min(8, 76 - nbits[t]);
             pos[t] = 76 - nbits[t] - w[t];
+            any_live = any_live || live[t];
         }
-        if (!live[0] && !live[1]) break;  // uniform: read from shared state after the barrier
+        if (!any_live) break;  // uniform: read from shared state after the barrier
         for (int b = tid; b < R; b += kRowRankThreads) {
             const u128 K = keyof(b);
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
+            for (int t = 0; t < NT; ++t) {
                 if (!live[t]) continue;
                 const int sh = 76 - nbits[t];
                 if (sh < 128 && (K >> sh) != (pre[t] >> sh)) continue;
@@ -524,7 +615,7 @@ __global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, l
             }
         }
         __syncthreads();
-        if (warp < 2 && live[warp]) {
+        if (warp < NT && live[warp]) {
             const int t = warp;
             // lane covers bins [255 - 8 lane - 7, 255 - 8 lane], descending
             const int top = 255 - 8 * lane;
@@ -556,37 +647,29 @@ __global__ void __launch_bounds__(kRowRankThreads) row_rank_kernel(PlanArgs p, l
         }
         __syncthreads();
     }
-    const u128 k8 = pre[0], kk = pre[1];
-    const bool has8 = T8 > 0, hask = Tk > 0;
+    const u128 k16 = pre[0], k8 = pre[1], kk = pre[2];
+    const bool has16 = C16 > 0, has8 = C8 > 0, hask = Ck > 0;
     for (int b = tid; b < R; b += kRowRankThreads) {
         const u128 K = keyof(b);
-        prec_s[b] = (has8 && K >= k8) ? 8 : ((hask && K >= kk) ? 4 : 0);
+        prec_s[b] = (has16 && K >= k16) ? 16 : (has8 && K >= k8) ? 8 : ((hask && K >= kk) ? 4 : 0);
     }
     __syncthreads();
     uint8_t* prow = p.prec + row * R;
     for (int b = tid; b < R; b += kRowRankThreads) prow[b] = prec_s[b];
     if (tid < 32) {
-        const unsigned lt = (1u << lane) - 1u;
-        uint16_t* krow = p.kidx + row * R;
-        int n8 = 0;
+        int n16 = 0, n8 = 0, n4 = 0;
         for (int b0 = 0; b0 < R; b0 += 32) {
             const int b = b0 + lane;
-            const bool is8 = b < R && prec_s[b] == 8;
-            const unsigned m = __ballot_sync(0xffffffffu, is8);
-            if (is8) krow[n8 + __popc(m & lt)] = (uint16_t)b;
-            n8 += __popc(m);
-        }
-        int n4 = 0;
-        for (int b0 = 0; b0 < R; b0 += 32) {
-            const int b = b0 + lane;
-            const bool is4 = b < R && prec_s[b] == 4;
-            const unsigned m = __ballot_sync(0xffffffffu, is4);
-            if (is4) krow[n8 + n4 + __popc(m & lt)] = (uint16_t)b;
-            n4 += __popc(m);
+            const int pr = b < R ? prec_s[b] : 0;
+            n16 += __popc(__ballot_sync(0xffffffffu, pr == 16));
+            n8 += __popc(__ballot_sync(0xffffffffu, pr == 8));
+            n4 += __popc(__ballot_sync(0xffffffffu, pr == 4));
         }
         if (lane == 0) {
-            p.cnt[row] = n8;
-            p.cnt[(size_t)p.BH * R + row] = n4;
+            const size_t BHRt = (size_t)p.BH * p.Rt, rt = (row / R) * p.Rt + row % R;
+            p.cnt[rt] = n8;
+            p.cnt[BHRt + rt] = n4;
+            p.cnt[2 * BHRt + rt] = n16 + p.Rp;  // every prefix key is kept at 16 bits
         }
     }
 }
@@ -599,9 +682,9 @@ size_t plan_scratch_bytes(int BH, int R) {
     size_t b = (size_t)BH * R * R * sizeof(double);        // max-branch logits
     b += (size_t)2 * BH * sizeof(unsigned long long);      // A bit range per head
     b = (b + 255) & ~(size_t)255;
-    b += (size_t)2 * BH * sizeof(SelectTarget);
+    b += (size_t)kTargets * BH * sizeof(SelectTarget);
     b = (b + 255) & ~(size_t)255;
-    b += (size_t)2 * BH * 4096 * sizeof(unsigned);
+    b += (size_t)kTargets * BH * 4096 * sizeof(unsigned);
     b = (b + 255) & ~(size_t)255;
     b += (size_t)BH * sizeof(unsigned);
     return b;
@@ -615,10 +698,10 @@ void plan_carve_scratch(PlanArgs* p, void* scratch) {
     off += (size_t)2 * p->BH * sizeof(unsigned long long);
     off = (off + 255) & ~(size_t)255;
     p->sel = reinterpret_cast<SelectTarget*>(c + off);
-    off += (size_t)2 * p->BH * sizeof(SelectTarget);
+    off += (size_t)kTargets * p->BH * sizeof(SelectTarget);
     off = (off + 255) & ~(size_t)255;
     p->hist = reinterpret_cast<unsigned*>(c + off);
-    off += (size_t)2 * p->BH * 4096 * sizeof(unsigned);
+    off += (size_t)kTargets * p->BH * 4096 * sizeof(unsigned);
     off = (off + 255) & ~(size_t)255;
     p->done_count = reinterpret_cast<unsigned*>(c + off);
 }
@@ -626,7 +709,9 @@ void plan_carve_scratch(PlanArgs* p, void* scratch) {
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     const int R = p.R, BH = p.BH;
     const long long RR = (long long)R * R;
-    const long long T8 = RR * p.bp8 / 10000, Tk = RR * (p.bp8 + p.bp4) / 10000;
+    // cumulative cuts of the ranking: 16-bit, 16+8-bit, kept
+    const long long C16 = RR * p.bp16 / 10000, C8 = RR * (p.bp16 + p.bp8) / 10000,
+                    Ck = RR * (p.bp16 + p.bp8 + p.bp4) / 10000;
     cudaError_t e;
     const double rd = 1.0 / sqrt((double)p.d);
     dim3 lg((R + kLgTile - 1) / kLgTile, (R + kLgTile - 1) / kLgTile, 2 * BH);
@@ -644,7 +729,8 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.abits_minmax, 0xFF, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(p.abits_minmax + BH, 0, sizeof(unsigned long long) * BH, stream)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(p.hist, 0, sizeof(unsigned) * 2 * 4096 * (size_t)BH, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p.hist, 0, sizeof(unsigned) * kTargets * 4096 * (size_t)BH, stream)) != cudaSuccess)
+        return e;
     if ((e = cudaMemsetAsync(p.done_count, 0, sizeof(unsigned) * (size_t)BH, stream)) != cudaSuccess) return e;
     const size_t smem = sizeof(double) * 2 * R;
     if (smem > 48 * 1024) {
@@ -653,24 +739,51 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     }
     softmax_kernel<<<(unsigned)((size_t)BH * R), kSoftThreads, smem, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // kept pairs of a head: the budgeted video pairs, plus every video row's
+    // prefix keys and every prefix row's keys
+    auto emit_lists = [&](long long budgeted) -> cudaError_t {
+        const long long per_head = budgeted + (long long)R * p.Rp + (long long)p.Rp * p.Rt;
+        offsets_kernel<<<(BH + 3) / 4, 128, 0, stream>>>(p, per_head);
+        lists_kernel<<<(unsigned)(((size_t)BH * p.Rt + 3) / 4), 128, 0, stream>>>(p);
+        return cudaGetLastError();
+    };
     if (p.per_row) {
         // ranking per query block: quotas per row, no selection passes
-        const long long T8r = (long long)R * p.bp8 / 10000, Tkr = (long long)R * (p.bp8 + p.bp4) / 10000;
-        row_rank_kernel<<<(unsigned)((size_t)BH * R), kRowRankThreads, 0, stream>>>(p, T8r, Tkr);
-        return cudaGetLastError();
+        const long long C16r = (long long)R * p.bp16 / 10000, C8r = (long long)R * (p.bp16 + p.bp8) / 10000,
+                        Ckr = (long long)R * (p.bp16 + p.bp8 + p.bp4) / 10000;
+        row_rank_kernel<<<(unsigned)((size_t)BH * R), kRowRankThreads, 0, stream>>>(p, C16r, C8r, Ckr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        return emit_lists((long long)R * Ckr);
     }
-    select_init_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(p, T8, Tk);
+    select_init_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(p, C16, C8, Ck);
     // about two 1024-thread CTAs per multiprocessor over all heads, so that
     // each CTA flushes its shared histogram once for many keys
     const long long per_head = std::max(1, 2 * std::max(1, p.num_sms) / BH);
     long long chunk = (RR + per_head - 1) / per_head;
     chunk = std::max<long long>(kHistMinChunk, (chunk + 4 * kHistThreads - 1) / (4 * kHistThreads) * (4 * kHistThreads));
     dim3 hg((unsigned)((RR + chunk - 1) / chunk), BH);
-    for (int pass = 0; pass < kSelectPasses; ++pass)
-        select_hist_kernel<<<hg, kHistThreads, 0, stream>>>(p, (int)chunk);
+    // with no 16-bit tier its (empty) target is skipped: two live targets
+    if (C16 > 0) {
+        constexpr size_t hs = 3 * 4096 * sizeof(unsigned);
+        if ((e = cudaFuncSetAttribute(select_hist_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hs)) !=
+            cudaSuccess)
+            return e;
+        for (int pass = 0; pass < kSelectPasses; ++pass)
+            select_hist_kernel<3><<<hg, kHistThreads, hs, stream>>>(p, (int)chunk);
+    } else {
+        for (int pass = 0; pass < kSelectPasses; ++pass)
+            select_hist_kernel<2><<<hg, kHistThreads, 2 * 4096 * sizeof(unsigned), stream>>>(p, (int)chunk);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     classify_kernel<<<(unsigned)(((size_t)BH * R + 3) / 4), 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return emit_lists(Ck);
+}
+
+long long plan_kept_per_head(int Rv, int Rp, int bp16, int bp8, int bp4, int per_row) {
+    const long long sum = bp16 + bp8 + bp4;
+    const long long budgeted = per_row ? (long long)Rv * ((long long)Rv * sum / 10000) : (long long)Rv * Rv * sum / 10000;
+    return budgeted + (long long)Rv * Rp + (long long)Rp * (Rv + Rp);
 }
 
 }  // namespace da2

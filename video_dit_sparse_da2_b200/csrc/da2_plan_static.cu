@@ -53,7 +53,7 @@ int static_scratch(da2_handle h, void** out) {
 }  // namespace
 
 extern "C" int da2_plan_static(da2_handle h, const da2_prepared* prep, const da2_budget* budget, uint8_t* prec,
-                               int32_t* cnt, uint16_t* kidx, double* A, void* stream) {
+                               int32_t* cnt, int64_t* off, uint16_t* kidx, double* A, void* stream) {
     if (!h) return DA2_ERR_ARG;
     da2_sizes_t sz;
     int rc = da2_sizes(h, &sz);
@@ -64,6 +64,7 @@ extern "C" int da2_plan_static(da2_handle h, const da2_prepared* prep, const da2
     da2_plan_bufs bufs;
     bufs.prec = prec;
     bufs.cnt = cnt;
+    bufs.off = off;
     bufs.kidx = kidx;
     bufs.A = A;
     bufs.scratch = scratch;

@@ -3,7 +3,8 @@
 //
 // One CTA per (64-token block a, head, tensor).  It gathers the block's
 // tokens through the partition (one coalesced 16-byte load per 8 channels of
-// a token row), then from the staged tile writes in a single pass:
+// a token row; all of a thread's loads are issued before the first is used),
+// then from the staged tile writes in a single pass:
 //   Q/K: pooled descriptors (fp64 mean over the valid slots, summed in slot
 //        order, and channel max; Eq. 2), FP8 e4m3 codes with the tile scale
 //        amax/448, two-level NVFP4 codes (tile scale amax/2688, ue4m3 scale
@@ -11,6 +12,9 @@
 //   V:   the transposed tile (V^T, value transposition folded into packing)
 //        quantized the same way with NVFP4 groups of 16 slots, and the
 //        per-head maxima of the V tile scales.
+// Optional extra outputs: the bf16 tiles of the 16-bit path (Q, K and V^T as
+// they are) and the INT8 tiles of the 8-bit phase's QK^T (Q and K; scale
+// amax/127, codes RNE(x * (127/amax)) clamped to +-127).
 // Operand tiles are written directly in the tcgen05 K-major no-swizzle
 // layout (core matrices of 8 rows x 16 bytes), so the attention kernel moves
 // each tile with one bulk copy.  Every quantizer step is an fp32
@@ -26,6 +30,11 @@ namespace {
 // threads per CTA: one quantization item (32 elements of an operand row) per thread
 template <int D>
 constexpr int threads_for() { return D == 64 ? 128 : 256; }
+// Resident CTAs per SM the register budget must allow: enough 16 KB tiles in
+// flight per SM to cover the memory latency (4 x 256 or 8 x 128 threads,
+// 64 registers each).
+template <int D>
+constexpr int min_ctas_for() { return D == 64 ? 8 : 4; }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a K-major
 // no-swizzle operand tile with `row_bytes` bytes per row: core matrices of
@@ -35,7 +44,7 @@ __device__ __forceinline__ uint32_t kmajor_offset(int row, int chunk, int row_by
 }
 
 template <int D>
-__global__ void __launch_bounds__(threads_for<D>()) prepare_kernel(PrepareArgs p) {
+__global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_kernel(PrepareArgs p) {
     constexpr int kThreads = threads_for<D>();
     constexpr int LD = D + 8;  // padded smem row (bf16 elements) against bank conflicts
     __shared__ __align__(16) uint16_t tile[64 * LD];
@@ -57,13 +66,21 @@ __global__ void __launch_bounds__(threads_for<D>()) prepare_kernel(PrepareArgs p
     const __nv_bfloat16* src = which == 0 ? p.q : (which == 1 ? p.k : p.v);
     src += (size_t)b * p.s0 + (size_t)h * p.s1;
     float amax = 0.0f;
-    for (int i = tid; i < 64 * (D / 8); i += kThreads) {
-        const int r = i / (D / 8), c8 = i % (D / 8);
+    constexpr int kChunks = 64 * (D / 8) / kThreads;  // 16-byte loads per thread
+    static_assert(kChunks * kThreads == 64 * (D / 8), "whole chunks per thread");
+    uint4 val[kChunks];
+#pragma unroll
+    for (int u = 0; u < kChunks; ++u) {
+        const int i = tid + u * kThreads, r = i / (D / 8), c8 = i % (D / 8);
         const int t = tok[r];
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (t >= 0) val = __ldg(reinterpret_cast<const uint4*>(src + (size_t)t * p.s2 + c8 * 8));
-        *reinterpret_cast<uint4*>(&tile[r * LD + c8 * 8]) = val;
-        const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+        val[u] = t >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)t * p.s2 + c8 * 8))
+                        : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kChunks; ++u) {
+        const int i = tid + u * kThreads, r = i / (D / 8), c8 = i % (D / 8);
+        *reinterpret_cast<uint4*>(&tile[r * LD + c8 * 8]) = val[u];
+        const uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             amax = fmaxf(amax, fabsf(__uint_as_float(w[e] << 16)));
@@ -100,10 +117,12 @@ __global__ void __launch_bounds__(threads_for<D>()) prepare_kernel(PrepareArgs p
     const float inv8 = zero ? 0.0f : __fdiv_rn(448.0f, amax);
     const float g4 = zero ? 0.0f : __fdiv_rn(amax, 2688.0f);
     const float t4 = zero ? 0.0f : __fdiv_rn(448.0f, amax);
+    const float inv8i = zero ? 0.0f : __fdiv_rn(127.0f, amax);
     if (tid == 0) {
         p.scale[(size_t)which * BH * R + ba] = s8;
         p.scale[(size_t)(3 + which) * BH * R + ba] = g4;
-        if (which == 2) {
+        if (p.si8 && which < 2) p.si8[(size_t)which * BH * R + ba] = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
+        if (which == 2 && a < p.Rv) {  // the phase units cover the video blocks
             atomicMax(reinterpret_cast<unsigned*>(&p.vmax[bh]), __float_as_uint(s8));
             atomicMax(reinterpret_cast<unsigned*>(&p.vmax[BH + bh]), __float_as_uint(g4));
         }
@@ -158,15 +177,40 @@ __global__ void __launch_bounds__(threads_for<D>()) prepare_kernel(PrepareArgs p
         for (int it = tid; it < 64 * (D / 32); it += kThreads) {
             const int r = it & 63, k = it >> 6;
             float x[32];
+            uint4 raw[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 w = *reinterpret_cast<const uint4*>(&tile[r * LD + 32 * k + 8 * q]);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                raw[q] = *reinterpret_cast<const uint4*>(&tile[r * LD + 32 * k + 8 * q]);
+                const uint32_t ww[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     x[8 * q + 2 * e] = bf_lo(ww[e]);
                     x[8 * q + 2 * e + 1] = bf_hi(ww[e]);
                 }
+            }
+            if (p.q16) {
+                // bf16 tile of the 16-bit path: the input values as they are (2D-byte rows)
+                uint8_t* dst16 = (which == 0 ? p.q16 : p.k16) + ba * (size_t)(128 * D);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(dst16 + kmajor_offset(r, 4 * k + q, 2 * D)) = raw[q];
+            }
+            if (p.q8i) {
+                int8_t* dsti = (which == 0 ? p.q8i : p.k8i) + ba * (size_t)(64 * D);
+                uint32_t wi[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    uint32_t acc = 0;
+#pragma unroll
+                    for (int b4 = 0; b4 < 4; ++b4) {
+                        int c = zero ? 0 : __float2int_rn(__fmul_rn(x[4 * e + b4], inv8i));
+                        c = c > 127 ? 127 : (c < -127 ? -127 : c);
+                        acc |= ((uint32_t)c & 0xFFu) << (8 * b4);
+                    }
+                    wi[e] = acc;
+                }
+                *reinterpret_cast<uint4*>(dsti + kmajor_offset(r, 2 * k, D)) = make_uint4(wi[0], wi[1], wi[2], wi[3]);
+                *reinterpret_cast<uint4*>(dsti + kmajor_offset(r, 2 * k + 1, D)) = make_uint4(wi[4], wi[5], wi[6], wi[7]);
             }
             *reinterpret_cast<uint4*>(dst8 + kmajor_offset(r, 2 * k, D)) = fp8x16(x);
             *reinterpret_cast<uint4*>(dst8 + kmajor_offset(r, 2 * k + 1, D)) = fp8x16(x + 16);
@@ -187,11 +231,29 @@ __global__ void __launch_bounds__(threads_for<D>()) prepare_kernel(PrepareArgs p
         for (int it = tid; it < (D / 2) * 4; it += kThreads) {
             const int c = it % (D / 2), k = it / (D / 2);
             float x0[16], x1[16];
+            uint32_t b16[2][8];  // bf16 pairs of V^T rows 2c and 2c+1 (slots 16k..16k+15)
 #pragma unroll
             for (int sl = 0; sl < 16; ++sl) {
                 const uint32_t w = *reinterpret_cast<const uint32_t*>(&tile[(16 * k + sl) * LD + 2 * c]);
                 x0[sl] = bf_lo(w);
                 x1[sl] = bf_hi(w);
+                if (sl & 1) {
+                    b16[0][sl >> 1] |= (w & 0xFFFFu) << 16;
+                    b16[1][sl >> 1] |= w & 0xFFFF0000u;
+                } else {
+                    b16[0][sl >> 1] = w & 0xFFFFu;
+                    b16[1][sl >> 1] = w >> 16;
+                }
+            }
+            if (p.v16) {
+                // bf16 V^T of the 16-bit path: rows 2c and 2c+1, 32 bytes each (128-byte rows)
+                uint8_t* dst16 = p.v16 + ba * (size_t)(128 * D);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q)
+                        *reinterpret_cast<uint4*>(dst16 + kmajor_offset(2 * c + hh, 2 * k + q, 128)) =
+                            make_uint4(b16[hh][4 * q], b16[hh][4 * q + 1], b16[hh][4 * q + 2], b16[hh][4 * q + 3]);
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {

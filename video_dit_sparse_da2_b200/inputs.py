@@ -27,10 +27,11 @@ class Workload:
     bp8: int   # basis points of the R^2 region pairs of a head kept in FP8
     bp4: int   # basis points kept in NVFP4; the rest are skipped
     lam: float = 0.2
+    P: int = 0  # prefix (text) tokens before the video tokens
 
     @property
     def N(self) -> int:
-        return self.F * self.Hv * self.Wv
+        return self.P + self.F * self.Hv * self.Wv
 
 
 # The five workload shapes (video latent geometry, head count and dim, budgets).
@@ -46,7 +47,12 @@ def wan14b(bp4: int) -> Workload:
 
 WAN14B_SWEEP = [wan14b(b) for b in (0, 2000, 4000, 6000)]
 ALL = [TINY, WAN13B, COGVIDEOX, HUNYUAN] + WAN14B_SWEEP
-BY_NAME = {w.name: w for w in ALL}
+# Shaped like the captured video-attention input of the pages' error analysis
+# (N = 109,376 tokens, 56 heads, d = 128, average-only draft guidance).  The
+# pages give no frame geometry: 256 prefix tokens + 31 frames of 44 x 80 is a
+# synthetic geometry with that token count.  Budgets: 10 / 30 / 60 %.
+CAPTURE = Workload("capture-shaped-109k", 1, 56, 128, 31, 44, 80, 1000, 3000, lam=0.0, P=256)
+BY_NAME = {w.name: w for w in ALL + [CAPTURE]}
 
 
 def make_qkv(B: int, H: int, N: int, d: int, seed: int = 0):

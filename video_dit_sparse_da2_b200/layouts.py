@@ -63,15 +63,42 @@ def prepared_to_logical(bufs: dict, B: int, H: int, R: int, d: int) -> dict:
     sc = g["scale"][: 6 * BH * R * 4].view(np.float32).reshape(6, B, H, R)
     out["s8"], out["g4"] = sc[:3], sc[3:]
     out["vmax"] = g["vmax"][: 2 * BH * 4].view(np.float32).reshape(2, B, H)
+    if "q8i" in g:
+        out["q8i"] = untile_kmajor(g["q8i"].reshape(B, H, R, 64 * d), 64, d).view(np.int8)
+        out["k8i"] = untile_kmajor(g["k8i"].reshape(B, H, R, 64 * d), 64, d).view(np.int8)
+        out["si8"] = g["si8"][: 2 * BH * R * 4].view(np.float32).reshape(2, B, H, R)
+    if "q16" in g:
+        # bf16 tiles of the 16-bit path, as uint16 bit patterns
+        def untile16(buf, rows, row_bytes):
+            return np.ascontiguousarray(untile_kmajor(buf.reshape(B, H, R, rows * row_bytes), rows,
+                                                      row_bytes)).view(np.uint16)
+        out["q16"] = untile16(g["q16"], 64, 2 * d)
+        out["k16"] = untile16(g["k16"], 64, 2 * d)
+        out["v16t"] = untile16(g["v16"], d, 128)
     return out
 
 
-def plan_to_logical(bufs: dict, B: int, H: int, R: int) -> dict:
+def plan_to_logical(bufs: dict, B: int, H: int, R: int, Rv: int = None) -> dict:
+    """Device plan buffers -> logical arrays; the compact lists are unpacked
+    into fixed-stride rows kidx[B,H,R,R] (entries past a row's count are 0).
+    R counts every block, Rv the video blocks (prec and A; default R)."""
+    Rv = R if Rv is None else Rv
     g = {k: v.cpu().numpy() for k, v in bufs.items() if k != "scratch"}
     BH = B * H
+    off = g["off"][: BH * (R + 1) * 8].view(np.int64).reshape(B, H, R + 1)
+    flat = g["kidx"].view(np.uint16)
+    kidx = np.zeros((B, H, R, R), np.uint16)
+    for b in range(B):
+        for h in range(H):
+            for a in range(R):
+                lo, hi = int(off[b, h, a]), int(off[b, h, a + 1])
+                kidx[b, h, a, : hi - lo] = flat[lo:hi]
     return {
-        "prec": g["prec"][: BH * R * R].reshape(B, H, R, R),
+        "prec": g["prec"][: BH * Rv * Rv].reshape(B, H, Rv, Rv),
         "cnt": g["cnt"][: 2 * BH * R * 4].view(np.int32).reshape(2, B, H, R),
-        "kidx": g["kidx"][: BH * R * R * 2].view(np.uint16).reshape(B, H, R, R),
-        "A": g["A"][: BH * R * R * 8].view(np.float64).reshape(B, H, R, R),
+        "cnt16": g["cnt"][2 * BH * R * 4: 3 * BH * R * 4].view(np.int32).reshape(B, H, R),
+        "off": off,
+        "kidx": kidx,
+        "kidx_flat": flat,
+        "A": g["A"][: BH * Rv * Rv * 8].view(np.float64).reshape(B, H, Rv, Rv),
     }

@@ -18,7 +18,7 @@ def main(argv=None) -> None:
     argv = sys.argv[1:] if argv is None else argv
     w = BY_NAME[argv[0] if argv else "wan2.1-1.3b-480p"]
     q, k, v = (t.cuda() for t in workload_qkv(w))
-    m = da2.DA2(w.B, w.H, w.d, w.F, w.Hv, w.Wv)
+    m = da2.DA2(w.B, w.H, w.d, w.F, w.Hv, w.Wv, w.P)
     out, prep, plan = m.forward(q, k, v, w.bp8, w.bp4, w.lam)
     m.attention(prep, plan, out)
     torch.cuda.synchronize()
