@@ -6,10 +6,11 @@
 // Work item = two query blocks (a0 = 2i, a1 = 2i+1) of one head stacked into
 // one M = 128 tile: the block-scaled NVFP4 MMA has M = 128 per CTA, the
 // method's query blocks have 64 tokens.  The kernel walks the union of the
-// two blocks' key lists, first all 8-bit key blocks (ascending), then all
-// 4-bit key blocks (ascending); a row takes part in a step only when its own
-// block kept that key block at that precision, so every row sees exactly its
-// own list in the order of the method.
+// two blocks' key lists phase by phase -- the 16-bit key blocks (when the
+// plan has any), then the 8-bit ones, then the 4-bit ones, each ascending; a
+// row takes part in a step only when its own block kept that key block at
+// that precision, so every row sees exactly its own list in the order of the
+// method.
 //
 // Roles (384 threads, two persistent CTAs per SM, each holding 256 of the 512
 // tensor-memory columns; items fetched from a global counter):
@@ -24,22 +25,25 @@
 //              group maximum of the scores) and e2m1 codes of p * (ratio *
 //              1/scale), the definition's (p * ratio) * 1/scale reordered,
 //              equal to it whenever p is a power of two; p of the winning key
-//              is exactly 1 in both -- and hands each row's factor for O (the
-//              running-max correction, times the change of units sigma8 ->
-//              sigma4 of Eq. 8 at the phase switch) to the correction warps.
-//              It never waits for the output accumulator.
-//   warps 4-7  correction: one thread per row, same lane quarters.  Before the
-//              PV of a step they wait for the previous PV and multiply their
-//              rows of O by the factor when any row of the warp needs it;
-//              at the end of an item they divide by l, convert to bf16 and
-//              store each row at its original token position.
+//              is exactly 1 in both; 16-bit: bf16 of p -- and, before the PV
+//              of a step, multiplies its row of O by the running-max
+//              correction times the change of units of Eq. 8 at a phase
+//              switch (after waiting for the previous PV), when any row of the
+//              warp needs it.  At the end of an item it hands each row's
+//              output scale (unit / l) to the epilogue warps.
+//   warps 4-7  epilogue: one thread per row, same lane quarters.  At the end
+//              of an item they multiply O by the output scale, convert to bf16
+//              and store each row at its original token position, while the
+//              softmax warps already work on the next item.
 //   warp 8     MMA issue (whole warp, one elected lane issues): S = Q K^T
-//              (tcgen05.mma kind::f8f6f4 or kind::mxf4nvf4 block16) into the S
-//              buffer, O += P V into the single O accumulator once the
-//              correction warps released the step.
+//              (tcgen05.mma kind::f8f6f4, kind::i8, kind::mxf4nvf4 block16 or
+//              kind::f16) into the S buffer, O += P V into the single O
+//              accumulator once the softmax warps published the step's P.
 //   warp 9     loader (whole warp, one elected lane issues): bulk async copies
 //              of the K / V tiles (pre-tiled by the preparation kernel) into a
 //              3-stage ring, and the step record of each stage.
+//   warps 10-11 scheduler: fetch the next work item and merge the two rows'
+//              lists into the item's step list.
 // Every mbarrier wait is bounded; a stuck wait sets the status word, all
 // roles drain their own outstanding work and the CTA frees tensor memory
 // before returning.
@@ -52,9 +56,9 @@ namespace {
 
 constexpr int kStages = 3;
 // Roles: softmax warps 0-3 (one thread per tile row, all 64 key columns of a
-// step), correction warps 4-7 (one thread per tile row), MMA warp 8, loader
-// warp 9; warps 10-11 complete the third warpgroup (the register budgets are
-// set per warpgroup of four warps) and only join the CTA barriers.
+// step), epilogue warps 4-7 (one thread per tile row), MMA warp 8, loader
+// warp 9, scheduler warps 10-11 (the register budgets are set per warpgroup
+// of four warps).
 constexpr int kSoftmaxThreads = 128;
 constexpr int kThreads = 384;
 constexpr int kMmaWarp = 8, kLoadWarp = 9;
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
     extern __shared__ __align__(1024) uint8_t smem[];
     // bar_empty[st] completes when the PV of a step in stage st has finished:
     // it frees the stage for the loader, frees that step's P buffer two steps
-    // later, and tells the correction warps that O holds the step.
+    // later, and tells the softmax and epilogue warps that O holds the step.
     __shared__ uint64_t bar_q, bar_qfree, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
         bar_epi, bar_osc[2], bar_drain, bar_ready[2], bar_listfree, bar_infofree[2];
     __shared__ uint32_t tmem_base_sh;
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
             mbar_init(&bar_p[s], 4);    // one arrive per softmax warp
             mbar_init(&bar_osc[s], 4);  // the softmax warps wrote an item's output scales
             mbar_init(&bar_ready[s], 1);      // the scheduler published an item
-            mbar_init(&bar_infofree[s], 4);   // the correction warps are done with an item
+            mbar_init(&bar_infofree[s], 4);   // the epilogue warps are done with an item
         }
         mbar_init(&bar_listfree, 6);  // loader, MMA warp and the four softmax warps read the list
         mbar_init(&bar_epi, 4);       // the epilogue warps read O of an item
@@ -304,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
     bool mma_issued = false;
 
     // Every role runs its own loop over the items the scheduler publishes; the
-    // warpgroups take their register budgets once, here: the correction and
+    // warpgroups take their register budgets once, here: the epilogue and
     // issue warpgroups release registers, the softmax warpgroup takes them
     // (a request blocks until the CTA's pool can serve it, with no time limit,
     // so only the softmax warpgroup ever requests before the end).
@@ -313,80 +317,80 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
         if (warp == kLoadWarp) {
             uint32_t gstep = 0;
             for (int k = 0;; ++k) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bar_ready[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns)))
-                        break;
-                    const int item = warp_uniform(info_sh[k & 1].item);
-                    if (item < 0) break;
-                    const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
-                      n_ent = warp_uniform(info_sh[k & 1].n_ent);
-                    const int bh = item / pairs, pr = item % pairs;
-                    const int a0 = 2 * pr, a1 = 2 * pr + 1;
-                    const bool has1 = a1 < R;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar_ready[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns)))
+                    break;
+                const int item = warp_uniform(info_sh[k & 1].item);
+                if (item < 0) break;
+                const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
+                  n_ent = warp_uniform(info_sh[k & 1].n_ent);
+                const int bh = item / pairs, pr = item % pairs;
+                const int a0 = 2 * pr, a1 = 2 * pr + 1;
+                const bool has1 = a1 < R;
 
-                    // ================================================== loader (whole warp, one elected lane issues)
-                    const size_t t0 = (size_t)bh * R + a0;
-                    const uint32_t qb8 = 64 * D, qb4 = 32 * D;
-                    const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
-                    // Q of this item replaces Q of the previous one once the previous
-                    // item's MMAs (which read it) have completed
-                    if (k > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar_qfree, (k - 1) & 1, abort_v, p.status, p.wait_ns)))
+                // ================================================== loader (whole warp, one elected lane issues)
+                const size_t t0 = (size_t)bh * R + a0;
+                const uint32_t qb8 = 64 * D, qb4 = 32 * D;
+                const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
+                // Q of this item replaces Q of the previous one once the previous
+                // item's MMAs (which read it) have completed
+                if (k > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar_qfree, (k - 1) & 1, abort_v, p.status, p.wait_ns)))
+                    break;
+                const uint32_t qb16 = T16 ? 128 * D : 0;
+                mbar_expect_tx_w(&bar_q, (has1 ? 2u : 1u) * (qb8 + qb4 + qb16));
+                // the 8-bit Q tile: INT8 codes when the 8-bit phase's QK^T is INT8
+                const uint8_t* q8src = p.q8i ? reinterpret_cast<const uint8_t*>(p.q8i) : p.q8;
+                bulk_g2s_w(smem + L::q8, q8src + t0 * qb8, qb8, &bar_q);
+                bulk_g2s_w(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
+                if constexpr (T16) bulk_g2s_w(smem + L::q16, p.q16 + t0 * qb16, qb16, &bar_q);
+                if (has1) {
+                    bulk_g2s_w(smem + L::q8 + qb8, q8src + (t0 + 1) * qb8, qb8, &bar_q);
+                    bulk_g2s_w(smem + L::q4 + qb4, p.q4 + (t0 + 1) * qb4, qb4, &bar_q);
+                    if constexpr (T16) bulk_g2s_w(smem + L::q16 + qb16, p.q16 + (t0 + 1) * qb16, qb16, &bar_q);
+                }
+                for (int j = 0; j < n_ent; ++j) {
+                    const uint32_t g = gstep + j, st = g % kStages;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status,
+                                                           p.wait_ns)))
                         break;
-                    const uint32_t qb16 = T16 ? 128 * D : 0;
-                    mbar_expect_tx_w(&bar_q, (has1 ? 2u : 1u) * (qb8 + qb4 + qb16));
-                    // the 8-bit Q tile: INT8 codes when the 8-bit phase's QK^T is INT8
-                    const uint8_t* q8src = p.q8i ? reinterpret_cast<const uint8_t*>(p.q8i) : p.q8;
-                    bulk_g2s_w(smem + L::q8, q8src + t0 * qb8, qb8, &bar_q);
-                    bulk_g2s_w(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
-                    if constexpr (T16) bulk_g2s_w(smem + L::q16, p.q16 + t0 * qb16, qb16, &bar_q);
-                    if (has1) {
-                        bulk_g2s_w(smem + L::q8 + qb8, q8src + (t0 + 1) * qb8, qb8, &bar_q);
-                        bulk_g2s_w(smem + L::q4 + qb4, p.q4 + (t0 + 1) * qb4, qb4, &bar_q);
-                        if constexpr (T16) bulk_g2s_w(smem + L::q16 + qb16, p.q16 + (t0 + 1) * qb16, qb16, &bar_q);
+                    const uint32_t e = warp_uniform((uint32_t)list[j]);
+                    const int kb = e & 0xFFF, ph = entry_phase(e);
+                    const size_t tk = (size_t)bh * R + kb;
+                    uint8_t* sb = smem + L::stage + st * L::stage_bytes;
+                    {
+                        // step record: lane i writes copy i (one 16-byte store per lane)
+                        // (the 16-bit path has no tile scales and unit 1)
+                        const int nk = p.n_a[kb];
+                        const float ck = ph == 2   ? 1.0f
+                                         : (ph == 0 && p.si8) ? p.si8[BHR + tk]
+                                                              : p.scale[(ph ? 4 : 1) * BHR + tk];
+                        const float vs = ph == 2 ? 1.0f : p.scale[(ph ? 5 : 2) * BHR + tk];
+                        const float sg = ph == 2 ? 1.0f : (ph ? sig4 : sig8);
+                        const float ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
+                        reinterpret_cast<uint4*>(smem + L::meta + st * 512)[lane] =
+                            make_uint4((uint32_t)nk, __float_as_uint(ck), __float_as_uint(ratio), 0u);
+                        // visible to the tensor-core copy of the MMA warp, which
+                        // waits on the arrive below
+                        fence_proxy_async_smem();
+                        __syncwarp();
                     }
-                    for (int j = 0; j < n_ent; ++j) {
-                        const uint32_t g = gstep + j, st = g % kStages;
-                        if (!__all_sync(0xffffffffu, mbar_wait(&bar_empty[st], ((g / kStages) & 1) ^ 1, abort_v, p.status,
-                                                               p.wait_ns)))
-                            break;
-                        const uint32_t e = warp_uniform((uint32_t)list[j]);
-                        const int kb = e & 0xFFF, ph = entry_phase(e);
-                        const size_t tk = (size_t)bh * R + kb;
-                        uint8_t* sb = smem + L::stage + st * L::stage_bytes;
-                        {
-                            // step record: lane i writes copy i (one 16-byte store per lane)
-                            // (the 16-bit path has no tile scales and unit 1)
-                            const int nk = p.n_a[kb];
-                            const float ck = ph == 2   ? 1.0f
-                                             : (ph == 0 && p.si8) ? p.si8[BHR + tk]
-                                                                  : p.scale[(ph ? 4 : 1) * BHR + tk];
-                            const float vs = ph == 2 ? 1.0f : p.scale[(ph ? 5 : 2) * BHR + tk];
-                            const float sg = ph == 2 ? 1.0f : (ph ? sig4 : sig8);
-                            const float ratio = sg > 0.0f ? __fdiv_rn(vs, sg) : 0.0f;
-                            reinterpret_cast<uint4*>(smem + L::meta + st * 512)[lane] =
-                                make_uint4((uint32_t)nk, __float_as_uint(ck), __float_as_uint(ratio), 0u);
-                            // visible to the tensor-core copy of the MMA warp, which
-                            // waits on the arrive below
-                            fence_proxy_async_smem();
-                            __syncwarp();
-                        }
-                        if (T16 && ph == 2) {
-                            mbar_expect_tx_w(&bar_full[st], 2 * 128 * D);
-                            bulk_g2s_w(sb + L::k_off, p.k16 + tk * (128 * D), 128 * D, &bar_full[st]);
-                            bulk_g2s_w(sb + L::v_off, p.v16 + tk * (128 * D), 128 * D, &bar_full[st]);
-                        } else if (ph == 0) {
-                            mbar_expect_tx_w(&bar_full[st], 2 * 64 * D);
-                            const uint8_t* k8src = p.k8i ? reinterpret_cast<const uint8_t*>(p.k8i) : p.k8;
-                            bulk_g2s_w(sb + L::k_off, k8src + tk * (64 * D), 64 * D, &bar_full[st]);
-                            bulk_g2s_w(sb + L::v_off, p.v8 + tk * (64 * D), 64 * D, &bar_full[st]);
-                        } else {
-                            mbar_expect_tx_w(&bar_full[st], 2 * 32 * D + 1024);
-                            bulk_g2s_w(sb + L::k_off, p.k4 + tk * (32 * D), 32 * D, &bar_full[st]);
-                            bulk_g2s_w(sb + L::v_off, p.v4 + tk * (32 * D), 32 * D, &bar_full[st]);
-                            bulk_g2s_w(sb + L::ksf_off, p.sfk + tk * 512, 512, &bar_full[st]);
-                            bulk_g2s_w(sb + L::vsf_off, p.sfv + tk * 512, 512, &bar_full[st]);
-                        }
-                        ++loads_issued;
+                    if (T16 && ph == 2) {
+                        mbar_expect_tx_w(&bar_full[st], 2 * 128 * D);
+                        bulk_g2s_w(sb + L::k_off, p.k16 + tk * (128 * D), 128 * D, &bar_full[st]);
+                        bulk_g2s_w(sb + L::v_off, p.v16 + tk * (128 * D), 128 * D, &bar_full[st]);
+                    } else if (ph == 0) {
+                        mbar_expect_tx_w(&bar_full[st], 2 * 64 * D);
+                        const uint8_t* k8src = p.k8i ? reinterpret_cast<const uint8_t*>(p.k8i) : p.k8;
+                        bulk_g2s_w(sb + L::k_off, k8src + tk * (64 * D), 64 * D, &bar_full[st]);
+                        bulk_g2s_w(sb + L::v_off, p.v8 + tk * (64 * D), 64 * D, &bar_full[st]);
+                    } else {
+                        mbar_expect_tx_w(&bar_full[st], 2 * 32 * D + 1024);
+                        bulk_g2s_w(sb + L::k_off, p.k4 + tk * (32 * D), 32 * D, &bar_full[st]);
+                        bulk_g2s_w(sb + L::v_off, p.v4 + tk * (32 * D), 32 * D, &bar_full[st]);
+                        bulk_g2s_w(sb + L::ksf_off, p.sfk + tk * 512, 512, &bar_full[st]);
+                        bulk_g2s_w(sb + L::vsf_off, p.sfv + tk * 512, 512, &bar_full[st]);
                     }
+                    ++loads_issued;
+                }
 
                 if (lane == 0) mbar_arrive(&bar_listfree);
                 gstep += n_ent;
@@ -394,125 +398,122 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
         } else if (warp == kMmaWarp) {
             uint32_t gstep = 0;
             for (int k = 0;; ++k) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bar_ready[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns)))
-                        break;
-                    const int item = warp_uniform(info_sh[k & 1].item);
-                    if (item < 0) break;
-                    const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
-                      n_ent = warp_uniform(info_sh[k & 1].n_ent);
-                    const int bh = item / pairs, pr = item % pairs;
-                    const int a0 = 2 * pr, a1 = 2 * pr + 1;
-                    const bool has1 = a1 < R;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar_ready[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns)))
+                    break;
+                const int item = warp_uniform(info_sh[k & 1].item);
+                if (item < 0) break;
+                const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
+                  n_ent = warp_uniform(info_sh[k & 1].n_ent);
 
-                    // ================================================== MMA issue (whole warp, one elected lane issues)
-                    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-                        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, p.status, p.wait_ns));
-                    };
-                    bool ok = wait_all(&bar_q, k & 1);
-                    ok = ok && wait_all(&bar_sfq, k & 1);
+                // ================================================== MMA issue (whole warp, one elected lane issues)
+                auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+                    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_v, p.status, p.wait_ns));
+                };
+                bool ok = wait_all(&bar_q, k & 1);
+                ok = ok && wait_all(&bar_sfq, k & 1);
+                tc_fence_after();
+                if (ok && n_ent > n16e + n8e) {
+                    for (int ch = 0; ch < D / 64; ++ch)
+                        tc_cp_32x128_x4_w(tmem + kColSfq + 4 * ch, sdesc(smem + L::sfq + 512 * ch, 128, 128));
+                }
+                // Descriptors of the fixed buffers; a stage or P buffer is selected
+                // by adding its byte offset / 16 to the start-address field (bits
+                // 0-13, which hold the shared-memory address / 16 without carry
+                // since shared memory ends below 256 KB).
+                const uint64_t dq8 = sdesc(smem + L::q8, 128, 8 * D), dq4 = sdesc(smem + L::q4, 128, 4 * D);
+                const uint64_t dst = sdesc(smem + L::stage, 0, 0);  // stage base: lbo / sbo added per operand
+                auto with_lbo_sbo = [](uint64_t d, uint32_t off, uint32_t lbo, uint32_t sbo) -> uint64_t {
+                    return d + (off >> 4) + ((uint64_t)(lbo >> 4) << 16) + ((uint64_t)(sbo >> 4) << 32);
+                };
+                const uint64_t dmeta = sdesc(smem + L::meta, 128, 128);
+                const bool qk_i8 = p.q8i != nullptr;  // the 8-bit phase's QK^T in INT8 (s32 scores)
+                const uint64_t dp8 = sdesc(smem + L::p, 128, 512), dp4 = sdesc(smem + L::p, 128, 256);
+                const uint64_t dpsf = sdesc(smem + L::p + L::p_sf, 128, 128);
+                auto issue_pv = [&](int i) -> bool {
+                    const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
+                    // P of step g is written (and O rescaled for it); the first PV of
+                    // an item overwrites O, which the epilogue of the previous item
+                    // must have read
+                    if (!wait_all(&bar_p[pb], (g >> 1) & 1)) return false;
+                    if (i == 0 && k > 0 && !wait_all(&bar_epi, (k - 1) & 1)) return false;
                     tc_fence_after();
-                    if (ok && n_ent > n16e + n8e) {
-                        for (int ch = 0; ch < D / 64; ++ch)
-                            tc_cp_32x128_x4_w(tmem + kColSfq + 4 * ch, sdesc(smem + L::sfq + 512 * ch, 128, 128));
+                    const int ph = entry_phase(warp_uniform((uint32_t)list[i]));
+                    const uint32_t so = st * L::stage_bytes;
+                    const uint64_t po = (pb * L::p_bytes) >> 4;
+                    if (T16 && ph == 2) {
+                        // bf16 P (128-byte rows) x bf16 V^T, K = 16 keys per MMA
+                        const uint64_t dp16 = sdesc(smem + L::p, 128, 1024);
+                        const uint64_t dv16 = with_lbo_sbo(dst, so + L::v_off, 128, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16_w(tmem + kColO, dp16 + po + 16 * kk, dv16 + 16 * kk, idesc_bf16(128, D),
+                                       (i > 0 || kk > 0) ? 1u : 0u);
+                    } else if (ph == 0) {
+                        const uint64_t dv8 = with_lbo_sbo(dst, so + L::v_off, 128, 512);
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk)
+                            mma_f8_w(tmem + kColO, dp8 + po + 16 * kk, dv8 + 16 * kk, idesc_f8(128, D),
+                                     (i > 0 || kk > 0) ? 1u : 0u);
+                    } else {
+                        tc_cp_32x128_x4_w(tmem + kColSfp + 4 * pb, dpsf + po);
+                        tc_cp_32x128_x4_w(tmem + kColSfv + 4 * pb, with_lbo_sbo(dst, so + L::vsf_off, 128, 128));
+                        mma_f4_w(tmem + kColO, dp4 + po, with_lbo_sbo(dst, so + L::v_off, 128, 256), idesc_f4(128, D),
+                                 tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
                     }
-                    // Descriptors of the fixed buffers; a stage or P buffer is selected
-                    // by adding its byte offset / 16 to the start-address field (bits
-                    // 0-13, which hold the shared-memory address / 16 without carry
-                    // since shared memory ends below 256 KB).
-                    const uint64_t dq8 = sdesc(smem + L::q8, 128, 8 * D), dq4 = sdesc(smem + L::q4, 128, 4 * D);
-                    const uint64_t dst = sdesc(smem + L::stage, 0, 0);  // stage base: lbo / sbo added per operand
-                    auto with_lbo_sbo = [](uint64_t d, uint32_t off, uint32_t lbo, uint32_t sbo) -> uint64_t {
-                        return d + (off >> 4) + ((uint64_t)(lbo >> 4) << 16) + ((uint64_t)(sbo >> 4) << 32);
-                    };
-                    const uint64_t dmeta = sdesc(smem + L::meta, 128, 128);
-                    const bool qk_i8 = p.q8i != nullptr;  // the 8-bit phase's QK^T in INT8 (s32 scores)
-                    const uint64_t dp8 = sdesc(smem + L::p, 128, 512), dp4 = sdesc(smem + L::p, 128, 256);
-                    const uint64_t dpsf = sdesc(smem + L::p + L::p_sf, 128, 128);
-                    auto issue_pv = [&](int i) -> bool {
-                        const uint32_t g = gstep + i, pb = g & 1, st = g % kStages;
-                        // P of step g is written (and O rescaled for it); the first PV of
-                        // an item overwrites O, which the epilogue of the previous item
-                        // must have read
-                        if (!wait_all(&bar_p[pb], (g >> 1) & 1)) return false;
-                        if (i == 0 && k > 0 && !wait_all(&bar_epi, (k - 1) & 1)) return false;
-                        tc_fence_after();
-                        const int ph = entry_phase(warp_uniform((uint32_t)list[i]));
-                        const uint32_t so = st * L::stage_bytes;
-                        const uint64_t po = (pb * L::p_bytes) >> 4;
-                        if (T16 && ph == 2) {
-                            // bf16 P (128-byte rows) x bf16 V^T, K = 16 keys per MMA
-                            const uint64_t dp16 = sdesc(smem + L::p, 128, 1024);
-                            const uint64_t dv16 = with_lbo_sbo(dst, so + L::v_off, 128, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_bf16_w(tmem + kColO, dp16 + po + 16 * kk, dv16 + 16 * kk, idesc_bf16(128, D),
-                                           (i > 0 || kk > 0) ? 1u : 0u);
-                        } else if (ph == 0) {
-                            const uint64_t dv8 = with_lbo_sbo(dst, so + L::v_off, 128, 512);
-#pragma unroll
-                            for (int kk = 0; kk < 2; ++kk)
-                                mma_f8_w(tmem + kColO, dp8 + po + 16 * kk, dv8 + 16 * kk, idesc_f8(128, D),
-                                         (i > 0 || kk > 0) ? 1u : 0u);
-                        } else {
-                            tc_cp_32x128_x4_w(tmem + kColSfp + 4 * pb, dpsf + po);
-                            tc_cp_32x128_x4_w(tmem + kColSfv + 4 * pb, with_lbo_sbo(dst, so + L::vsf_off, 128, 128));
-                            mma_f4_w(tmem + kColO, dp4 + po, with_lbo_sbo(dst, so + L::v_off, 128, 256), idesc_f4(128, D),
-                                     tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
-                        }
-                        // frees the stage and (two steps later) the P buffer, and tells
-                        // the correction warps that O holds step g
-                        tc_commit_w(&bar_empty[st]);
-                        return true;
-                    };
-                    for (int j = 0; j < n_ent && ok; ++j) {
-                        const uint32_t g = gstep + j, st = g % kStages;
-                        if (!wait_all(&bar_full[st], (g / kStages) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        // the S buffer is free once every softmax warp has read step g-1
-                        if (g > 0 && !wait_all(&bar_sfree, (g - 1) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const int ph = entry_phase(warp_uniform((uint32_t)list[j]));
-                        const uint32_t so = st * L::stage_bytes;
-                        const uint32_t sd = tmem + kColS;
-                        // step record next to S (the previous one was read with S(g-1))
-                        tc_cp_32x128_x4_w(tmem + kColMeta, dmeta + st * (512 >> 4));
-                        if (T16 && ph == 2) {
-                            // bf16 Q (2D-byte rows) x bf16 K, K = 16 channels per MMA
-                            const uint64_t dq16 = sdesc(smem + L::q16, 128, 16 * D);
-                            const uint64_t dk16 = with_lbo_sbo(dst, so + L::k_off, 128, 16 * D);
-#pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                mma_bf16_w(sd, dq16 + 16 * kk, dk16 + 16 * kk, idesc_bf16(128, 64), kk > 0 ? 1u : 0u);
-                        } else if (ph == 0) {
-                            const uint64_t dk8 = with_lbo_sbo(dst, so + L::k_off, 128, 8 * D);
-#pragma unroll
-                            for (int kk = 0; kk < D / 32; ++kk) {
-                                if (qk_i8)
-                                    mma_i8_w(sd, dq8 + 16 * kk, dk8 + 16 * kk, idesc_i8(128, 64), kk > 0 ? 1u : 0u);
-                                else
-                                    mma_f8_w(sd, dq8 + 16 * kk, dk8 + 16 * kk, idesc_f8(128, 64), kk > 0 ? 1u : 0u);
-                            }
-                        } else {
-                            tc_cp_32x128_x4_w(tmem + kColSfk, with_lbo_sbo(dst, so + L::ksf_off, 128, 128));
-                            const uint64_t dk4 = with_lbo_sbo(dst, so + L::k_off, 128, 4 * D);
-#pragma unroll
-                            for (int kk = 0; kk < D / 64; ++kk)
-                                mma_f4_w(sd, dq4 + 16 * kk, dk4 + 16 * kk, idesc_f4(128, 64), tmem + kColSfq + 4 * kk,
-                                         tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
-                        }
-                        tc_commit_w(&bar_s);
-                        mma_issued = true;
-                        if (j > 0 && !issue_pv(j - 1)) {
-                            ok = false;
-                            break;
-                        }
+                    // frees the stage and (two steps later) the P buffer, and tells
+                    // the softmax and epilogue warps that O holds step g
+                    tc_commit_w(&bar_empty[st]);
+                    return true;
+                };
+                for (int j = 0; j < n_ent && ok; ++j) {
+                    const uint32_t g = gstep + j, st = g % kStages;
+                    if (!wait_all(&bar_full[st], (g / kStages) & 1)) {
+                        ok = false;
+                        break;
                     }
-                    if (ok && n_ent > 0) ok = issue_pv(n_ent - 1);
+                    // the S buffer is free once every softmax warp has read step g-1
+                    if (g > 0 && !wait_all(&bar_sfree, (g - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int ph = entry_phase(warp_uniform((uint32_t)list[j]));
+                    const uint32_t so = st * L::stage_bytes;
+                    const uint32_t sd = tmem + kColS;
+                    // step record next to S (the previous one was read with S(g-1))
+                    tc_cp_32x128_x4_w(tmem + kColMeta, dmeta + st * (512 >> 4));
+                    if (T16 && ph == 2) {
+                        // bf16 Q (2D-byte rows) x bf16 K, K = 16 channels per MMA
+                        const uint64_t dq16 = sdesc(smem + L::q16, 128, 16 * D);
+                        const uint64_t dk16 = with_lbo_sbo(dst, so + L::k_off, 128, 16 * D);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_bf16_w(sd, dq16 + 16 * kk, dk16 + 16 * kk, idesc_bf16(128, 64), kk > 0 ? 1u : 0u);
+                    } else if (ph == 0) {
+                        const uint64_t dk8 = with_lbo_sbo(dst, so + L::k_off, 128, 8 * D);
+#pragma unroll
+                        for (int kk = 0; kk < D / 32; ++kk) {
+                            if (qk_i8)
+                                mma_i8_w(sd, dq8 + 16 * kk, dk8 + 16 * kk, idesc_i8(128, 64), kk > 0 ? 1u : 0u);
+                            else
+                                mma_f8_w(sd, dq8 + 16 * kk, dk8 + 16 * kk, idesc_f8(128, 64), kk > 0 ? 1u : 0u);
+                        }
+                    } else {
+                        tc_cp_32x128_x4_w(tmem + kColSfk, with_lbo_sbo(dst, so + L::ksf_off, 128, 128));
+                        const uint64_t dk4 = with_lbo_sbo(dst, so + L::k_off, 128, 4 * D);
+#pragma unroll
+                        for (int kk = 0; kk < D / 64; ++kk)
+                            mma_f4_w(sd, dq4 + 16 * kk, dk4 + 16 * kk, idesc_f4(128, 64), tmem + kColSfq + 4 * kk,
+                                     tmem + kColSfk + 2 * kk, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit_w(&bar_s);
+                    mma_issued = true;
+                    if (j > 0 && !issue_pv(j - 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (ok && n_ent > 0) ok = issue_pv(n_ent - 1);
 
                 // Q of this item is free once its MMAs have completed
                 tc_commit_w(&bar_qfree);
@@ -525,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
             // union of the two rows' lists per phase
             const int stid = tid - 10 * 32;
             for (int k = 0;; ++k) {
-                // the list of item k-1 has been read, and the correction warps
+                // the list of item k-1 has been read, and the epilogue warps
                 // are done with the item record of item k-2
                 bool ok = true;
                 if (k > 0) ok = mbar_wait(&bar_listfree, (k - 1) & 1, abort_v, p.status, p.wait_ns);
