@@ -63,8 +63,8 @@ typedef struct {
     int F, Hv, Wv; /* frames and latent frame size */
     int C;         /* region capacity = attention block size; must be 64 */
     int P;         /* prefix (text) tokens before the video tokens, 0 = none;
-                      N = P + F*Hv*Wv tokens.  Prefix interactions lie outside
-                      the precision budget (App. C.1): video queries keep every
+                      N = P + F*Hv*Wv tokens.  Pairs with a prefix block are not
+                      counted in the precision budget (App. C.1): video queries keep every
                       prefix key and prefix queries attend to every key, on the
                       16-bit path (which then needs the bf16 operands). */
 } da2_shape;
@@ -74,8 +74,8 @@ typedef struct {
     int bp_fp4;    /* basis points kept in NVFP4; bp_fp16 + bp_fp8 + bp_fp4 <= 10000; the rest
                       is skipped */
     double lambda; /* max-pool branch weight of the draft map (Eq. 3); 0 = average only */
-    int per_row;   /* 0: rank all R^2 pairs of a head (DraftAttention2, Sec. 3.1 and App. C.1
-                      "ranks all video-region pairs within each head").  1: rank the R key
+    int per_row;   /* 0: rank all R^2 pairs of a head together (DraftAttention2, Sec. 3.1
+                      and App. C.1: one ranking per head).  1: rank the R key
                       blocks of each query block separately, quotas floor(R bp/10^4) per row
                       (a reading of a per-query-row ranking; ties to the smaller key block). */
     int bp_fp16;   /* basis points kept at 16 bits (bf16 operands; Table 1's 16-bit share),

@@ -260,8 +260,8 @@ int oracle_partition(int Hv, int Wv, int C, int* region_of, int* slot_of, int* n
 /* ------------------------------------------------------------------------ */
 /* Shapes and the token <-> slot tables.                                     */
 /* ------------------------------------------------------------------------ */
-/* Prefix (text) tokens, App. C.1 ("Prefix interactions lie outside the     */
-/* video-region budget").  Reading of the sequence layout, which the pages  */
+/* Prefix (text) tokens, App. C.1: the precision budget counts only pairs  */
+/* of video regions.  Reading of the sequence layout, which the pages       */
 /* do not give: the P prefix tokens come first (positions 0..P-1), the      */
 /* video tokens follow in raster order (P + f*Hv*Wv + y*Wv + x).  The       */
 /* prefix is packed into Rp = ceil(P/64) blocks of consecutive tokens, which */
@@ -515,9 +515,9 @@ int oracle_prepare(int B, int H, int d, int F, int Hv, int Wv, const uint16_t* q
 }
 
 /* ------------------------------------------------------------------------ */
-/* 5b. INT8 operands of the paper's 8-bit QK^T (App. C.1: "The INT8 path    */
-/* uses INT8 for QK^T and FP8 for the probability-value multiplication";    */
-/* the scale placement is a reading, as for FP8): per 64-token tile         */
+/* 5b. INT8 operands of the paper's 8-bit QK^T (App. C.1: its 8-bit path   */
+/* multiplies Q and K in INT8 and keeps P V in FP8; the scale placement is  */
+/* a reading, as for FP8): per 64-token tile                                */
 /* s = amax/127 (fp32 divide), code = clamp(RNE(x * (127/amax)), -127, 127) */
 /* with the product rounded in fp32; dequantized value = code * s; a zero   */
 /* tile has s = 0 and all-zero codes.                                        */
@@ -737,9 +737,9 @@ int oracle_assign_tiers(int BH, int R, const double* A, int bp16, int bp8, int b
 }
 
 /* ------------------------------------------------------------------------ */
-/* 4d. Prefix keys and queries (App. C.1: "video queries retain all valid    */
-/* prefix keys, and prefix queries use non-sparse attention"; "Prefix        */
-/* interactions lie outside the video-region budget").  Reading of the      */
+/* 4d. Prefix keys and queries (App. C.1: a video query keeps every valid  */
+/* prefix key, a prefix query attends to every key, and neither kind of     */
+/* pair counts against the video-region budget).  Reading of the            */
 /* unstated precision: both run on the 16-bit path, the reference precision */
 /* (the budget that assigns the lower precisions covers only video-region   */
 /* pairs).  From a video plan (cnt [3][BH][Rv], lists [BH][Rv][Rv] of item  */

@@ -1,6 +1,6 @@
-"""GPU parity of the prefix (text) tokens (DraftAttention2 App. C.1: prefix
-interactions lie outside the video-region budget; video queries keep all valid
-prefix keys; prefix queries use non-sparse attention): slot tables, the plan
+"""GPU parity of the prefix (text) tokens (DraftAttention2 App. C.1: the budget
+covers video-region pairs only; every video query block also sees every valid
+prefix key and every prefix query sees all keys): slot tables, the plan
 (precision map of the video pairs, counts, offsets and lists over every block)
 bit for bit, and the attention within the output tolerance of the oracle."""
 import numpy as np

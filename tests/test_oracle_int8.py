@@ -1,5 +1,5 @@
-"""Pins of the oracle's INT8 QK^T path (DraftAttention2 App. C.1: "The INT8
-path uses INT8 for QK^T and FP8 for the probability-value multiplication").
+"""Pins of the oracle's INT8 QK^T path (DraftAttention2 App. C.1: the 8-bit
+path computes Q K^T from INT8 operands and P V from FP8 ones).
 Reading of the unstated scale: symmetric per 64-token tile, s = amax/127,
 code = clamp(RNE(x * (127/amax)), -127, 127), zero tile -> s = 0, codes 0.
 """

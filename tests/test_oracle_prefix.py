@@ -1,6 +1,6 @@
-"""Pins of the oracle's prefix (text) tokens (DraftAttention2 App. C.1: prefix
-interactions lie outside the video-region budget; video queries retain all
-valid prefix keys; prefix queries use non-sparse attention).  Readings: the P
+"""Pins of the oracle's prefix (text) tokens (DraftAttention2 App. C.1: the
+budget covers video-region pairs only; every video query block also sees every
+valid prefix key and every prefix query sees all keys).  Readings: the P
 prefix tokens come first in the sequence and are packed into ceil(P/64) blocks
 after the video blocks; prefix interactions run on the 16-bit path.
 """
