@@ -29,13 +29,11 @@ sys.path.insert(0, ROOT)
 METRIC = "ms/call and dense-equiv TFLOPS at 1 B200; % of mixed FP8/FP4 tensor roofline"
 
 # DRAM bytes (read + write) of one attention launch, measured by ncu
-# (dram__bytes_read.sum + dram__bytes_write.sum) for the attention sources whose
-# hash is given; any other source or workload reports null.  Filled in only from
-# a capture of the current kernel.  HunyuanVideo-720p: a capture of the same
-# geometry with 4 of the 24 heads (167,016,192 + 86,479,872 bytes), times 6 for
-# the heads of a full launch (heads are independent work items).
+# (dram__bytes_read.sum + dram__bytes_write.sum, one pass, full-size launch) for
+# the attention sources whose hash is given; any other source or workload
+# reports null.  Filled in only from a capture of the current kernel.
 ATTN_TRAFFIC: dict = {
-    "hunyuanvideo-720p": {"bytes": 6 * (167016192 + 86479872), "sources_sha256_16": "79ed505beaddd851"},
+    "hunyuanvideo-720p": {"bytes": 998.90e6 + 698.16e6, "sources_sha256_16": "79ed505beaddd851"},
 }
 _ATTN_SOURCES = ("video_dit_sparse_da2_b200/csrc/da2_attention.cu", "video_dit_sparse_da2_b200/csrc/da2_common.cuh")
 
