@@ -76,17 +76,17 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
         val[u] = t >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)t * p.s2 + c8 * 8))
                         : make_uint4(0, 0, 0, 0);
     }
+    // |x| of a finite bf16 orders like its 15 magnitude bits, so the tile
+    // maximum is taken on the bits, two halves per instruction
+    uint32_t mag2 = 0u;
 #pragma unroll
     for (int u = 0; u < kChunks; ++u) {
         const int i = tid + u * kThreads, r = i / (D / 8), c8 = i % (D / 8);
         *reinterpret_cast<uint4*>(&tile[r * LD + c8 * 8]) = val[u];
-        const uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[e] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[e] & 0xFFFF0000u)));
-        }
+        mag2 = __vmaxu2(mag2, __vmaxu2(val[u].x & 0x7FFF7FFFu, val[u].y & 0x7FFF7FFFu));
+        mag2 = __vmaxu2(mag2, __vmaxu2(val[u].z & 0x7FFF7FFFu, val[u].w & 0x7FFF7FFFu));
     }
+    amax = __uint_as_float(max(mag2 & 0xFFFFu, mag2 >> 16) << 16);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
@@ -97,18 +97,25 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
 
     auto X = [&](int r, int c) -> float { return bf16_bits_to_f32(tile[r * LD + c]); };
 
-    // ---- pooled descriptors (Eq. 2), Q and K only
-    if (which < 2 && tid < D) {
+    // ---- pooled descriptors (Eq. 2), Q and K only: thread c < D sums column c
+    // in fp64 in slot order, thread D + c takes its maximum (exact in fp32, the
+    // values are bf16), so each thread runs one dependency chain
+    static_assert(kThreads >= 2 * D, "a sum thread and a max thread per channel");
+    if (which < 2 && tid < 2 * D) {
         const int na = p.n_a[a];
-        double s = 0.0, m = (double)X(0, tid);
-        for (int j = 0; j < na; ++j) {
-            const double x = (double)X(j, tid);
-            s += x;
-            m = fmax(m, x);
-        }
+        const int c = tid < D ? tid : tid - D;
         const size_t plane = (size_t)BH * R * D;
-        p.desc[(2 * which) * plane + ba * D + tid] = s / (double)na;
-        p.desc[(2 * which + 1) * plane + ba * D + tid] = m;
+        if (tid < D) {
+            double s = 0.0;
+#pragma unroll 8
+            for (int j = 0; j < na; ++j) s += (double)X(j, c);
+            p.desc[(2 * which) * plane + ba * D + c] = s / (double)na;
+        } else {
+            float m = X(0, c);
+#pragma unroll 8
+            for (int j = 1; j < na; ++j) m = fmaxf(m, X(j, c));
+            p.desc[(2 * which + 1) * plane + ba * D + c] = (double)m;
+        }
     }
 
     // ---- scales
@@ -139,9 +146,12 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
     auto fp8x16 = [&](const float* x) -> uint4 {
         uint32_t w[4];
 #pragma unroll
+        const float2 s2 = make_float2(inv8, inv8);
         for (int e = 0; e < 4; ++e) {
-            const uint16_t lo = zero ? 0 : cvt_e4m3x2(__fmul_rn(x[4 * e], inv8), __fmul_rn(x[4 * e + 1], inv8));
-            const uint16_t hi = zero ? 0 : cvt_e4m3x2(__fmul_rn(x[4 * e + 2], inv8), __fmul_rn(x[4 * e + 3], inv8));
+            const float2 y0 = __fmul2_rn(make_float2(x[4 * e], x[4 * e + 1]), s2);
+            const float2 y1 = __fmul2_rn(make_float2(x[4 * e + 2], x[4 * e + 3]), s2);
+            const uint16_t lo = zero ? 0 : cvt_e4m3x2(y0.x, y0.y);
+            const uint16_t hi = zero ? 0 : cvt_e4m3x2(y1.x, y1.y);
             w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
         }
         return make_uint4(w[0], w[1], w[2], w[3]);
@@ -151,19 +161,21 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
     auto fp4x16 = [&](const float* x, uint8_t* sf_out) -> uint2 {
         float a16 = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a16 = fmaxf(a16, fabsf(x[e]));
+        for (int e = 0; e < 16; e += 2) a16 = max3f(a16, fabsf(x[e]), fabsf(x[e + 1]));
         const uint32_t sf = zero ? 0u : (uint32_t)(cvt_e4m3x2(__fmul_rn(a16, t4), 0.0f) & 0xFF);
         *sf_out = (uint8_t)sf;
         if (sf == 0) return make_uint2(0u, 0u);
         const float rcp = __frcp_rn(__fmul_rn(e4m3_to_f32((uint8_t)sf), g4));
+        const float2 r2 = make_float2(rcp, rcp);
         uint32_t w[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t acc = 0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                acc |= (uint32_t)cvt_e2m1x2(__fmul_rn(x[8 * h + 2 * e], rcp), __fmul_rn(x[8 * h + 2 * e + 1], rcp))
-                       << (8 * e);
+            for (int e = 0; e < 4; ++e) {
+                const float2 y = __fmul2_rn(make_float2(x[8 * h + 2 * e], x[8 * h + 2 * e + 1]), r2);
+                acc |= (uint32_t)cvt_e2m1x2(y.x, y.y) << (8 * e);
+            }
             w[h] = acc;
         }
         return make_uint2(w[0], w[1]);
