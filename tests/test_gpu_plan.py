@@ -67,3 +67,23 @@ def test_plan_bit_exact_wan13b():
     q, k, v = inputs(B, H, d, F, Hv, Wv)
     A = O.draft(O.prepare(q, k, v, F, Hv, Wv).desc, 0.2)
     _check_plan(res["plan"], A, O.assign(A, 1000, 3000))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_plan_max_branch_exact_path_and_fp64_fallback(d):
+    # The max-pool branch's logits of blocks whose channel maxima span at most
+    # a few binades come from exact integer tensor-core products, the others
+    # from the fp64 chain; both must give the defining fp64 values.  Frames 0-1
+    # (Q) and 5 (K) get one channel scaled by 2^-10, which widens those blocks'
+    # range past the exact one; frame 7 gets an all-negative Q channel (a
+    # negative maximum); R = 300 spans three 128-block tiles, mixing tiles with
+    # and without such blocks.
+    B, H, F, Hv, Wv = 1, 2, 12, 30, 52
+    q, k, v = make_qkv(B, H, F * Hv * Wv, d, seed=4)
+    fr = Hv * Wv
+    q[:, :, 0:2 * fr, 0] *= 2.0 ** -10
+    k[:, :, 5 * fr:6 * fr, 3] *= 2.0 ** -10
+    q[:, :, 7 * fr:8 * fr, 2] = -(q[:, :, 7 * fr:8 * fr, 2].abs() + 1.0)
+    res = gpu_run(B, H, d, F, Hv, Wv, 1000, 3000, qkv=(q, k, v))
+    A = O.draft(O.prepare(q, k, v, F, Hv, Wv).desc, 0.2)
+    _check_plan(res["plan"], A, O.assign(A, 1000, 3000))

@@ -194,7 +194,7 @@ int da2_sizes(da2_handle h, da2_sizes_t* o) {
     o->off = BH * (R + 1) * sizeof(int64_t);
     o->kidx = BH * R * R * sizeof(uint16_t);
     o->A = BH * Rv * Rv * sizeof(double);
-    o->plan_scratch = da2::plan_scratch_bytes((int)BH, (int)Rv);
+    o->plan_scratch = da2::plan_scratch_bytes((int)BH, (int)Rv, h->shape.d);
     o->q16 = o->k16 = o->v16 = BH * R * 128 * d;
     o->q8i = o->k8i = BH * R * 64 * d;
     o->si8 = 2 * BH * R * sizeof(float);
@@ -275,6 +275,7 @@ int da2_plan(da2_handle h, const da2_prepared* prep, const da2_budget* budget, c
     a.kidx = plan->kidx;
     a.status = h->d_status;
     a.num_sms = h->num_sms;
+    a.wait_ns = h->wait_ns;
     da2::plan_carve_scratch(&a, plan->scratch);
     cudaError_t e = da2::launch_plan(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DA2_OK : cuda_fail(e);

@@ -67,6 +67,12 @@ __global__ void __launch_bounds__(kLgThreads, 1) logits_kernel(PlanArgs p, doubl
     double* sK = lg_smem + 2 * kLgKc * kLgTile;    // [2][kLgKc][kLgTile]
     const int R = p.R, bh = blockIdx.z >> 1, branch = blockIdx.z & 1;
     const int a0 = blockIdx.y * kLgTile, b0 = blockIdx.x * kLgTile;
+    // max-pool branch: a tile whose query and key blocks are all inside the
+    // exact range was written by the integer tensor-core path (same values)
+    if (branch == 1) {
+        const size_t nt = (size_t)p.mx_rpad / kLgTile;
+        if (p.mx_tile_ok[(size_t)bh * nt + blockIdx.y] && p.mx_tile_ok[((size_t)p.BH + bh) * nt + blockIdx.x]) return;
+    }
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
     // descriptors of every block are stored (Rt per head); the draft uses the
     // R video blocks
@@ -678,7 +684,7 @@ constexpr int kSelectPasses = 8;  // 12-bit digits cover the 96-bit key
 
 }  // namespace
 
-size_t plan_scratch_bytes(int BH, int R) {
+size_t plan_scratch_bytes(int BH, int R, int d) {
     size_t b = (size_t)BH * R * R * sizeof(double);        // max-branch logits
     b += (size_t)2 * BH * sizeof(unsigned long long);      // A bit range per head
     b = (b + 255) & ~(size_t)255;
@@ -687,6 +693,8 @@ size_t plan_scratch_bytes(int BH, int R) {
     b += (size_t)kTargets * BH * 4096 * sizeof(unsigned);
     b = (b + 255) & ~(size_t)255;
     b += (size_t)BH * sizeof(unsigned);
+    b = (b + 255) & ~(size_t)255;
+    b += mx_scratch_bytes(BH, R, d);  // split descriptors of the exact max-pool branch
     return b;
 }
 
@@ -704,6 +712,9 @@ void plan_carve_scratch(PlanArgs* p, void* scratch) {
     off += (size_t)kTargets * p->BH * 4096 * sizeof(unsigned);
     off = (off + 255) & ~(size_t)255;
     p->done_count = reinterpret_cast<unsigned*>(c + off);
+    off += (size_t)p->BH * sizeof(unsigned);
+    off = (off + 255) & ~(size_t)255;
+    mx_carve(p, c + off);
 }
 
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
@@ -714,6 +725,10 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
                     Ck = RR * (p.bp16 + p.bp8 + p.bp4) / 10000;
     cudaError_t e;
     const double rd = 1.0 / sqrt((double)p.d);
+    // the max-pool branch's logits of every block inside the exact range come
+    // from integer tensor-core products; the fp64 chain below covers the rest
+    if (mx_tile_rows() != kLgTile) return cudaErrorInvalidValue;  // both paths share the 128-block tiles
+    if ((e = launch_max_logits(p, rd, stream)) != cudaSuccess) return e;
     dim3 lg((R + kLgTile - 1) / kLgTile, (R + kLgTile - 1) / kLgTile, 2 * BH);
     if (p.d == 64) {
         if ((e = cudaFuncSetAttribute(logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLgSmem)) !=
