@@ -30,6 +30,11 @@ constexpr int kMxTile = 128;     // rows per split tile (the MMA's M)
 constexpr int kMxN = 64;         // key blocks per MMA tile (the MMA's N)
 constexpr uint32_t kMxCols = 256;  // tensor-memory columns: HH, HL + LH, LL (3 x 64 used)
 constexpr int kMxThreads = 128;
+// dynamic shared memory: hi / lo tiles of A (128 rows) and B (64 rows), then
+// the epilogue's staging rows (4 warps x 32 x 33 doubles)
+template <int D>
+constexpr int stage_off() { return 384 * D; }
+constexpr int kStageBytes = 4 * 32 * 33 * 8;
 
 __device__ __forceinline__ uint32_t kmajor_off_b(int row, int byte, int row_bytes) {
     return ((row >> 3) * (row_bytes >> 4) + (byte >> 4)) * 128 + (row & 7) * 16 + (byte & 15);
@@ -190,24 +195,33 @@ __global__ void __launch_bounds__(kMxThreads) mx_logits_kernel(PlanArgs p, doubl
     const int e0a = a < R ? p.mx_e0[ra] : 0;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     if (__all_sync(0xffffffffu, done)) {
-        double* orow = p.Lmax + ((size_t)bh * R + (a < R ? a : 0)) * R;
+        // each warp stages its 32 rows x 32 columns in shared memory (rows
+        // padded to 33 doubles against bank conflicts), then writes them row by
+        // row, 32 consecutive key blocks per store
+        double* stage = reinterpret_cast<double*>(sm + stage_off<D>()) + warp * 32 * 33;
 #pragma unroll 1
         for (int c0 = 0; c0 < kMxN; c0 += 32) {
             uint32_t hh[32], hx[32], ll[32];
             tmem_ld32(lane_base + c0, hh);
             tmem_ld32(lane_base + 64 + c0, hx);
             tmem_ld32(lane_base + 128 + c0, ll);
-            if (oka) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int b = b0 + c0 + j;
-                    if (b >= R || !okb_sh[c0 + j]) continue;
-                    const long long T = ((long long)(int)hh[j] << 14) + ((long long)(int)hx[j] << 7) + (long long)(int)ll[j];
-                    const int s = e0a + e0b_sh[c0 + j] - 14;  // within the normal range: |s| < 300
-                    const double scale = __longlong_as_double((long long)(s + 1023) << 52);
-                    orow[b] = ((double)T * scale) * rd;
-                }
+            for (int j = 0; j < 32; ++j) {
+                const long long T = ((long long)(int)hh[j] << 14) + ((long long)(int)hx[j] << 7) + (long long)(int)ll[j];
+                const int s = e0a + e0b_sh[c0 + j] - 14;  // within the normal range: |s| < 300
+                const double scale = __longlong_as_double((long long)(s + 1023) << 52);
+                stage[lane * 33 + j] = ((double)T * scale) * rd;
             }
+            __syncwarp();
+            const int b = b0 + c0 + lane;
+            const bool okc = b < R && okb_sh[c0 + lane];
+#pragma unroll 4
+            for (int r = 0; r < 32; ++r) {
+                const int ar = a0 + 32 * warp + r;
+                const bool okr = __shfl_sync(0xffffffffu, oka, r);
+                if (okr && okc) p.Lmax[((size_t)bh * R + ar) * R + b] = stage[r * 33 + lane];
+            }
+            __syncwarp();
         }
     } else if (threadIdx.x == 0 && issued) {
         // the MMAs did not complete within the limit: wait for them before
@@ -257,9 +271,11 @@ cudaError_t launch_max_logits(const PlanArgs& p, double rd, cudaStream_t stream)
     if (e != cudaSuccess) return e;
     dim3 sg((Rp + 7) / 8, 2, BH);
     dim3 lg((p.R + kMxN - 1) / kMxN, Rp / kMxTile, BH);
-    // at least 80 KB per CTA so that no more than two CTAs (2 x 256 of the 512
-    // tensor-memory columns) share a multiprocessor
-    const int smem = 80 * 1024;
+    // 84 KB per CTA: the tiles and the epilogue's staging rows, and more than a
+    // third of the multiprocessor's shared memory, so that no more than two
+    // CTAs (2 x 256 of the 512 tensor-memory columns) share a multiprocessor
+    static_assert(384 * 128 + kStageBytes <= 84 * 1024, "tiles and staging fit");
+    const int smem = 84 * 1024;
     if (p.d == 64) {
         mx_split_kernel<64><<<sg, 256, 0, stream>>>(p);
         if ((e = cudaFuncSetAttribute(mx_logits_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
