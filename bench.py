@@ -153,7 +153,8 @@ def run_ours(args, w, rank, world):
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(dev)
     m = da2.DA2(w.B, w.H, w.d, w.F, w.Hv, w.Wv)
-    qh, kh, vh = (t.pin_memory() for t in workload_qkv(w, seed=0))
+    structured = args.inputs == "structured"
+    qh, kh, vh = (t.pin_memory() for t in workload_qkv(w, seed=1 if structured else 0, structured=structured))
     q, k, v = (t.to(dev) for t in (qh, kh, vh))
     prep = m.alloc_prepared(dev)
     plan = m.alloc_plan(dev, (w.bp8, w.bp4))
@@ -270,19 +271,22 @@ def run_ours(args, w, rank, world):
 class OracleSampler:
     """Times the oracle on bounded samples of one call of workload w.
 
-    The inputs (the same seeded tensors as the device run, restricted to the
-    first `hs` heads, hs = min(H, host threads)) are drawn once.  A sample
+    The inputs (the device run's recipe and seed with `hs` heads, hs =
+    min(H, host threads)) are drawn once.  A sample
     runs prepare + draft + assign on those heads and attention on a doubling
     number of random query blocks per head until its time budget is used;
     the per-call time is extrapolated linearly to all heads and blocks."""
 
-    def __init__(self, w):
+    def __init__(self, w, structured=False):
         from oracle import oracle as O
-        from video_dit_sparse_da2_b200.inputs import make_qkv
+        from video_dit_sparse_da2_b200.inputs import make_qkv, make_qkv_structured
         self.O, self.w = O, w
         self.cores = O.num_threads()
         self.hs = max(1, min(w.H, self.cores))
-        self.qkv = make_qkv(w.B, self.hs, w.N, w.d, seed=0)
+        if structured:
+            self.qkv = make_qkv_structured(w.B, self.hs, w.d, w.F, w.Hv, w.Wv, w.P, seed=1)
+        else:
+            self.qkv = make_qkv(w.B, self.hs, w.N, w.d, seed=0)
         self.rng = __import__("numpy").random.default_rng(0)
 
     def sample(self, budget_s: float):
@@ -325,6 +329,8 @@ def main():
     ap.add_argument("--workload", default="hunyuanvideo-720p")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # the i.i.d. set (headline) or the structured second set (smooth per-frame field on Q, K)
+    ap.add_argument("--inputs", default="iid", choices=["iid", "structured"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -338,6 +344,7 @@ def main():
               "N": w.N, "budget_fp8_fp4_skip_pct": [w.bp8 / 100, w.bp4 / 100, 100 - (w.bp8 + w.bp4) / 100],
               "lambda": w.lam, "global_batch": w.B * world, "seq_len": w.N,
               "parallelism": f"replicas x{world} (independent calls, no collective)",
+              "inputs": "i.i.d. N(0,1), seed 0" if args.inputs == "iid" else "structured (smooth per-frame field on Q, K), seed 1",
               "l2": f"inputs larger than L2 ({3 * w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB of bf16 Q/K/V read per step)"}
 
     if args.impl == "reference":
@@ -346,7 +353,7 @@ def main():
         # inputs drawn once; one short untimed sample loads the oracle, then K
         # timed samples of about 60 s of CPU work in total; the line reports
         # their median
-        sampler = OracleSampler(w)
+        sampler = OracleSampler(w, structured=args.inputs == "structured")
         sampler.sample(budget_s=0.5)
         per = max(2.0, 60.0 / max(1, args.steps))
         runs = [sampler.sample(budget_s=per) for _ in range(args.steps)]
@@ -356,7 +363,7 @@ def main():
         value = flops / t_call / 1e12
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_call * 1e3, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": ("synthetic (seeded N(0,1) bf16)" if args.inputs == "iid" else "synthetic (seeded N(0,1) bf16 plus a smooth per-frame field on Q and K)"),
                 "config": config,
                 "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -390,7 +397,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8-e4m3 + nvfp4-e2m1 MMAs (bf16 in/out, fp64 draft)", "data": "synthetic (seeded N(0,1) bf16)",
+        "dtype": "fp8-e4m3 + nvfp4-e2m1 MMAs (bf16 in/out, fp64 draft)", "data": ("synthetic (seeded N(0,1) bf16)" if args.inputs == "iid" else "synthetic (seeded N(0,1) bf16 plus a smooth per-frame field on Q and K)"),
         "config": config,
         "ms_per_call": {"prepare": r["t_prep"], "plan": r["t_plan"], "attention": r["t_attn"], "total": ms},
         "roofline": {"bound": "tensor", "kernel": "attention", "achieved": achieved, "peak": peak_mix,
@@ -417,7 +424,7 @@ def main():
                            "peak_gbs": peaks["hbm_gbs"],
                            "frac": prep_bytes / (r["t_prep"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     if world == 1 and not args.no_cpu_baseline:
-        sampler = OracleSampler(w)
+        sampler = OracleSampler(w, structured=args.inputs == "structured")
         t_call, sample = sampler.sample(budget_s=20.0)
         line["cpu_baseline"] = {"value": flops / t_call / 1e12, "unit": UNIT, "cores": sampler.cores,
                                 "kind": "oracle", "sample": sample}

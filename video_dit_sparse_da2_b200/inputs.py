@@ -7,9 +7,17 @@ use it, so that both sides see the same bf16 tensors.
 Recipe: Q, K, V ~ i.i.d. N(0, 1), drawn in float32 with a CPU
 ``torch.Generator`` seeded with ``seed``, in the order Q, K, V, each of
 shape [B, H, N, d], then rounded to bf16 (round to nearest even).
+
+Second, structured set (``make_qkv_structured``, seed 1): the same i.i.d.
+draw, then Q and K (video tokens only) get an added smooth per-frame field,
+x += 2 f(frame, y/Hv, x/Wv), where per (batch, head, channel) f is half the sum
+of 4 cosines of low spatial frequency (integer wave numbers 0..2 along each
+axis, random phase) whose phases drift slowly from frame to frame; the draft
+map of such inputs is far from uniform, like that of video latents.
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass
 
 import torch
@@ -65,5 +73,32 @@ def make_qkv(B: int, H: int, N: int, d: int, seed: int = 0):
     return tuple(out)
 
 
-def workload_qkv(w: Workload, seed: int = 0):
+def make_qkv_structured(B: int, H: int, d: int, F: int, Hv: int, Wv: int, P: int = 0, seed: int = 1):
+    """bf16 Q, K, V of shape [B, H, P + F*Hv*Wv, d] on the CPU: the second,
+    structured input set of the module docstring."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    N = P + F * Hv * Wv
+    qkv = [torch.randn((B, H, N, d), generator=g, dtype=torch.float32) for _ in range(3)]
+    xx = (torch.arange(Wv, dtype=torch.float32) / Wv).view(1, 1, 1, Wv)
+    yy = (torch.arange(Hv, dtype=torch.float32) / Hv).view(1, 1, Hv, 1)
+    for t in qkv[:2]:
+        kx = torch.randint(0, 3, (B, H, 4, d), generator=g).float()
+        ky = torch.randint(0, 3, (B, H, 4, d), generator=g).float()
+        ph = torch.rand((B, H, 4, d), generator=g) * (2 * math.pi)
+        dr = (torch.rand((B, H, 4, d), generator=g) - 0.5) * 0.2
+        for b in range(B):
+            for h in range(H):
+                # spatial phase [4, d, Hv, Wv]
+                sp = 2 * math.pi * (kx[b, h, :, :, None, None] * xx + ky[b, h, :, :, None, None] * yy) \
+                    + ph[b, h, :, :, None, None]
+                for f in range(F):
+                    field = 0.5 * torch.cos(sp + dr[b, h, :, :, None, None] * f).sum(0)  # [d, Hv, Wv]
+                    t[b, h, P + f * Hv * Wv:P + (f + 1) * Hv * Wv, :] += 2.0 * field.reshape(d, Hv * Wv).T
+    return tuple(x.to(torch.bfloat16) for x in qkv)
+
+
+def workload_qkv(w: Workload, seed: int = 0, structured: bool = False):
+    if structured:
+        return make_qkv_structured(w.B, w.H, w.d, w.F, w.Hv, w.Wv, w.P, seed)
     return make_qkv(w.B, w.H, w.N, w.d, seed)
