@@ -19,6 +19,8 @@ struct da2_ctx {
     std::vector<int32_t> slot_token, n_a;  // host copies
     int32_t* d_slot_token = nullptr;       // [Npad]
     int32_t* d_n_a = nullptr;              // [R]
+    int32_t* d_pairs = nullptr;            // [npairs][2] query blocks sharing an attention tile (-1: none)
+    int npairs = 0;
     unsigned* d_status = nullptr;          // kernel status word
     int* d_work = nullptr;                 // attention work counter
     unsigned long long wait_ns = DA2_WAIT_NS_DEFAULT;  // limit of the kernels' bounded waits
@@ -131,8 +133,31 @@ int da2_create(const da2_shape* s, da2_handle* out) {
         h->n_a[a] = cnt;
         for (int j = 0; j < cnt; ++j) h->slot_token[(size_t)a * 64 + j] = 64 * i + j;
     }
+    // Query blocks that share one 128-row attention tile: block j of frame 2f
+    // with block j of frame 2f + 1 (the same patch one frame later, whose key
+    // lists are most alike in video, so the tile's merged list is shortest);
+    // the blocks of a last, unpaired frame and the prefix blocks pair with
+    // their successors.
+    std::vector<int32_t> pairs;
+    for (int f = 0; f + 1 < s->F; f += 2)
+        for (int j = 0; j < part.Rf; ++j) {
+            pairs.push_back(f * part.Rf + j);
+            pairs.push_back((f + 1) * part.Rf + j);
+        }
+    auto successive = [&](int base, int n) {
+        for (int i = 0; i < n; i += 2) {
+            pairs.push_back(base + i);
+            pairs.push_back(i + 1 < n ? base + i + 1 : -1);
+        }
+    };
+    if (s->F % 2) successive((s->F - 1) * part.Rf, part.Rf);
+    successive(h->Rv, h->Rp);
+    h->npairs = (int)(pairs.size() / 2);
     if ((e = cudaMalloc(&h->d_slot_token, sizeof(int32_t) * h->Npad)) != cudaSuccess ||
         (e = cudaMalloc(&h->d_n_a, sizeof(int32_t) * h->R)) != cudaSuccess ||
+        (e = cudaMalloc(&h->d_pairs, sizeof(int32_t) * pairs.size())) != cudaSuccess ||
+        (e = cudaMemcpy(h->d_pairs, pairs.data(), sizeof(int32_t) * pairs.size(), cudaMemcpyHostToDevice)) !=
+            cudaSuccess ||
         (e = cudaMalloc(&h->d_status, sizeof(unsigned))) != cudaSuccess ||
         (e = cudaMalloc(&h->d_work, sizeof(int))) != cudaSuccess ||
         (e = cudaMemcpy(h->d_slot_token, h->slot_token.data(), sizeof(int32_t) * h->Npad, cudaMemcpyHostToDevice)) !=
@@ -167,6 +192,7 @@ int da2_destroy(da2_handle h) {
     if (!h) return DA2_OK;
     cudaFree(h->d_slot_token);
     cudaFree(h->d_n_a);
+    cudaFree(h->d_pairs);
     cudaFree(h->d_status);
     cudaFree(h->d_work);
     delete h;
@@ -305,6 +331,8 @@ int da2_attention(da2_handle h, const da2_prepared* prep, const da2_plan_bufs* p
     a.cnt = plan->cnt;
     a.off = reinterpret_cast<const long long*>(plan->off);
     a.kidx = plan->kidx;
+    a.pairs = h->d_pairs;
+    a.npairs = h->npairs;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.o0 = out_strides[0];
     a.o1 = out_strides[1];

@@ -3,9 +3,10 @@
 // "Cross-precision accumulation" Eq. 8; App. B.3 shared normalization;
 // App. C.1 formats and empty rows).
 //
-// Work item = two query blocks (a0 = 2i, a1 = 2i+1) of one head stacked into
-// one M = 128 tile: the block-scaled NVFP4 MMA has M = 128 per CTA, the
-// method's query blocks have 64 tokens.  The kernel walks the union of the
+// Work item = two query blocks (a0, a1) of one head stacked into one M = 128
+// tile: the block-scaled NVFP4 MMA has M = 128 per CTA, the method's query
+// blocks have 64 tokens.  The pairs come from the handle's table (the same
+// patch in two consecutive frames, whose lists are most alike in video).  The kernel walks the union of the
 // two blocks' key lists phase by phase -- the 16-bit key blocks (when the
 // plan has any), then the 8-bit ones, then the 4-bit ones, each ascending; a
 // row takes part in a step only when its own block kept that key block at
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
     const int tid = threadIdx.x, warp = warp_uniform(tid >> 5), lane = tid & 31;
     const int R = p.R, BH = p.B * p.H;
     const size_t BHR = (size_t)BH * R;
-    const int pairs = (R + 1) / 2;
+    const int pairs = p.npairs;
     const int items = BH * pairs;
     const int nwords = (R + 31) / 32;
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + L::bitmap);
@@ -324,11 +325,11 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                 const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
                   n_ent = warp_uniform(info_sh[k & 1].n_ent);
                 const int bh = item / pairs, pr = item % pairs;
-                const int a0 = 2 * pr, a1 = 2 * pr + 1;
-                const bool has1 = a1 < R;
+                const int a0 = p.pairs[2 * pr], a1 = p.pairs[2 * pr + 1];
+                const bool has1 = a1 >= 0;
 
                 // ================================================== loader (whole warp, one elected lane issues)
-                const size_t t0 = (size_t)bh * R + a0;
+                const size_t t0 = (size_t)bh * R + a0, t1 = (size_t)bh * R + (has1 ? a1 : a0);
                 const uint32_t qb8 = 64 * D, qb4 = 32 * D;
                 const float sig8 = __fdiv_rn(p.vmax[bh], 448.0f), sig4 = __fdiv_rn(p.vmax[BH + bh], 2688.0f);
                 // Q of this item replaces Q of the previous one once the previous
@@ -343,9 +344,9 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                 bulk_g2s_w(smem + L::q4, p.q4 + t0 * qb4, qb4, &bar_q);
                 if constexpr (T16) bulk_g2s_w(smem + L::q16, p.q16 + t0 * qb16, qb16, &bar_q);
                 if (has1) {
-                    bulk_g2s_w(smem + L::q8 + qb8, q8src + (t0 + 1) * qb8, qb8, &bar_q);
-                    bulk_g2s_w(smem + L::q4 + qb4, p.q4 + (t0 + 1) * qb4, qb4, &bar_q);
-                    if constexpr (T16) bulk_g2s_w(smem + L::q16 + qb16, p.q16 + (t0 + 1) * qb16, qb16, &bar_q);
+                    bulk_g2s_w(smem + L::q8 + qb8, q8src + t1 * qb8, qb8, &bar_q);
+                    bulk_g2s_w(smem + L::q4 + qb4, p.q4 + t1 * qb4, qb4, &bar_q);
+                    if constexpr (T16) bulk_g2s_w(smem + L::q16 + qb16, p.q16 + t1 * qb16, qb16, &bar_q);
                 }
                 for (int j = 0; j < n_ent; ++j) {
                     const uint32_t g = gstep + j, st = g % kStages;
@@ -544,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                     break;
                 }
                 const int bh = item / pairs, pr = item % pairs;
-                const int a0 = 2 * pr, a1 = 2 * pr + 1;
-                const bool has1 = a1 < R;
+                const int a0 = p.pairs[2 * pr], a1 = p.pairs[2 * pr + 1];
+                const bool has1 = a1 >= 0;
                 constexpr int nph = T16 ? 3 : 2;  // phases 0 (8-bit), 1 (4-bit), 2 (16-bit)
                 for (int i = stid; i < 2 * nph * nwords; i += 64) bitmap[i] = 0u;
                 sched_barrier();
@@ -621,15 +622,15 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                 const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
                       n_ent = warp_uniform(info_sh[k & 1].n_ent);
                 const int bh = item / pairs, pr = item % pairs;
-                const int a0 = 2 * pr, a1 = 2 * pr + 1;
-                const bool has1 = a1 < R;
+                const int a0 = p.pairs[2 * pr], a1 = p.pairs[2 * pr + 1];
+                const bool has1 = a1 >= 0;
 
                 // ================================================== softmax
                 const int quarter = warp;                       // tensor-memory lane quarter
                 const int r = 32 * quarter + lane;              // tile row
                 const int hf = quarter >> 1;                    // which query block of the pair (= r >> 6)
-                const int a = hf ? a1 : a0;
                 const bool qvalid = hf == 0 || has1;
+                const int a = qvalid && hf ? a1 : a0;
                 const size_t ta = (size_t)bh * R + (qvalid ? a : a0);
                 const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
                 const float rdl2e = (D == 64 ? 0.125f : 0.0883883461356163025f) * 1.4426950408889634f;
@@ -910,15 +911,15 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                 const int n16e = warp_uniform(info_sh[k & 1].n16e), n8e = warp_uniform(info_sh[k & 1].n8e),
                       n_ent = warp_uniform(info_sh[k & 1].n_ent);
                 const int bh = item / pairs, pr = item % pairs;
-                const int a0 = 2 * pr, a1 = 2 * pr + 1;
-                const bool has1 = a1 < R;
+                const int a0 = p.pairs[2 * pr], a1 = p.pairs[2 * pr + 1];
+                const bool has1 = a1 >= 0;
 
                 // ================================================== epilogue
                 const int quarter = warp - 4;
                 const int r = 32 * quarter + lane;
                 const int hf = quarter >> 1;
-                const int a = hf ? a1 : a0;
                 const bool qvalid = hf == 0 || has1;
+                const int a = qvalid && hf ? a1 : a0;
                 const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
                 // the softmax warps' output scales of this item
                 bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_osc[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns));
@@ -1034,7 +1035,7 @@ cudaError_t launch_d(const AttnArgs& p, int items, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_attention(const AttnArgs& p, cudaStream_t stream) {
-    const int items = p.B * p.H * ((p.R + 1) / 2);
+    const int items = p.B * p.H * p.npairs;
     if (items == 0) return cudaSuccess;
     cudaError_t e = cudaMemsetAsync(p.work_counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;

@@ -85,6 +85,8 @@ struct AttnArgs {
     int B, H, d, R, N;
     const int32_t* slot_token;  // [64 R]
     const int32_t* n_a;         // [R]
+    const int32_t* pairs;       // [npairs][2] query blocks of each work item's tile (second -1: none)
+    int npairs;
     const uint8_t *q8, *k8, *v8, *q4, *k4, *v4, *sfq, *sfk, *sfv;
     const uint8_t *q16, *k16, *v16;  // bf16 tiles of the 16-bit path, or all null
     const int8_t *q8i, *k8i;         // INT8 Q/K tiles: the 8-bit phase's QK^T in INT8, or null
