@@ -391,9 +391,10 @@ def main():
     t_att = r["t_attn"] * 1e-3
     achieved = (F8 + F4) / t_att / 1e12
     peak_mix = (F8 + F4) / t_roof / 1e12 if t_roof > 0 else None
-    # prepare; max-pool split and integer logits, fp64 logits, softmax,
-    # selection init, 8 selection passes, classify, list offsets, lists; attention
-    launches_per_step = 1 + (2 + 1 + 1 + 1 + 8 + 1 + 1 + 1) + 1
+    # prepare; max-pool split, integer logits and fp64 strips, fp64 logits,
+    # softmax, selection init, 8 selection passes, classify, list offsets, lists;
+    # attention
+    launches_per_step = 1 + (3 + 1 + 1 + 1 + 8 + 1 + 1 + 1) + 1
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -65,16 +65,15 @@ struct PlanArgs {
     int num_sms;             // multiprocessors of the device (grid sizing)
     unsigned long long wait_ns;  // limit of the bounded device waits
     // max-pool branch from exact integer tensor-core products (scratch):
-    int8_t* mx_tiles;        // [2][BH][Rpad/128][hi, lo][128 * d] split descriptors, K-major
+    int8_t* mx_tiles;        // [2][BH][Rpad/128][3 parts][128 * d] split descriptors, K-major
     int* mx_e0;              // [2][BH][Rpad] smallest exponent of each block
     uint8_t* mx_ok;          // [2][BH][Rpad] block inside the exact range
-    uint8_t* mx_tile_ok;     // [2][BH][Rpad/128] every block of the 128-block tile inside it
+    int* mx_fail;            // [1 + 2 BH Rpad]: count, then (t BH + bh) Rpad + r of each block outside it
     int mx_rpad;             // R rounded up to 128
 };
 size_t plan_scratch_bytes(int BH, int R, int d);
 size_t mx_scratch_bytes(int BH, int R, int d);
 void mx_carve(PlanArgs* p, char* c);
-int mx_tile_rows();
 cudaError_t launch_max_logits(const PlanArgs& p, double rd, cudaStream_t stream);
 // Kept pairs of one head under a budget (the length of its part of kidx).
 long long plan_kept_per_head(int Rv, int Rp, int bp16, int bp8, int bp4, int per_row);

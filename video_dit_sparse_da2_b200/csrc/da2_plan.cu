@@ -67,12 +67,9 @@ __global__ void __launch_bounds__(kLgThreads, 1) logits_kernel(PlanArgs p, doubl
     double* sK = lg_smem + 2 * kLgKc * kLgTile;    // [2][kLgKc][kLgTile]
     const int R = p.R, bh = blockIdx.z >> 1, branch = blockIdx.z & 1;
     const int a0 = blockIdx.y * kLgTile, b0 = blockIdx.x * kLgTile;
-    // max-pool branch: a tile whose query and key blocks are all inside the
-    // exact range was written by the integer tensor-core path (same values)
-    if (branch == 1) {
-        const size_t nt = (size_t)p.mx_rpad / kLgTile;
-        if (p.mx_tile_ok[(size_t)bh * nt + blockIdx.y] && p.mx_tile_ok[((size_t)p.BH + bh) * nt + blockIdx.x]) return;
-    }
+    // the max-pool branch comes from the exact integer tensor-core path and
+    // its fp64 strips (launch_max_logits)
+    if (branch == 1) return;
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
     // descriptors of every block are stored (Rt per head); the draft uses the
     // R video blocks
@@ -727,7 +724,6 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream) {
     const double rd = 1.0 / sqrt((double)p.d);
     // the max-pool branch's logits of every block inside the exact range come
     // from integer tensor-core products; the fp64 chain below covers the rest
-    if (mx_tile_rows() != kLgTile) return cudaErrorInvalidValue;  // both paths share the 128-block tiles
     if ((e = launch_max_logits(p, rd, stream)) != cudaSuccess) return e;
     dim3 lg((R + kLgTile - 1) / kLgTile, (R + kLgTile - 1) / kLgTile, 2 * BH);
     if (p.d == 64) {
