@@ -26,16 +26,20 @@
 //              group maximum of the scores) and e2m1 codes of p * (ratio *
 //              1/scale), the definition's (p * ratio) * 1/scale reordered,
 //              equal to it whenever p is a power of two; p of the winning key
-//              is exactly 1 in both; 16-bit: bf16 of p -- and, before the PV
-//              of a step, multiplies its row of O by the running-max
+//              is exactly 1 in both; 16-bit: bf16 of p.  Once the row max of
+//              a step is known it posts the row's factor for O (running-max
 //              correction times the change of units of Eq. 8 at a phase
-//              switch (after waiting for the previous PV), when any row of the
-//              warp needs it.  At the end of an item it hands each row's
-//              output scale (unit / l) to the epilogue warps.
-//   warps 4-7  epilogue: one thread per row, same lane quarters.  At the end
-//              of an item they multiply O by the output scale, convert to bf16
-//              and store each row at its original token position, while the
-//              softmax warps already work on the next item.
+//              switch) to the correction warp of its quarter.  At the end of
+//              an item it hands each row's output scale (unit / l) to the
+//              epilogue.
+//   warps 4-7  correction and epilogue: one thread per row, same lane
+//              quarters.  Per step they multiply the rows of O whose factor is
+//              not 1 (after the previous PV has completed), off the softmax
+//              warps' path; the step's PV waits for them and for the softmax
+//              warps.  At the end of an item they multiply O by the output
+//              scale, convert to bf16 and store each row at its original token
+//              position, while the softmax warps already work on the next
+//              item.
 //   warp 8     MMA issue (whole warp, one elected lane issues): S = Q K^T
 //              (tcgen05.mma kind::f8f6f4, kind::i8, kind::mxf4nvf4 block16 or
 //              kind::f16) into the S buffer, O += P V into the single O
@@ -218,31 +222,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-// 64 consecutive 32-bit columns of this warp's lanes: two 32-column loads in
-// flight and one wait (no single instruction wider than 32 registers).
-__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr, uint32_t (&r)[64]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
-        "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]),
-          "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]),
-          "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
-          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
-          "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr), "r"(taddr + 32)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st32x2(uint32_t taddr, const uint32_t (&r)[64]) {
-    tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
-    tmem_st32(taddr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&r[32]));
-}
-
 template <int D, bool T16>
 __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnArgs p) {
     using L = Smem<D, T16>;
@@ -251,12 +230,13 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
     // it frees the stage for the loader, frees that step's P buffer two steps
     // later, and tells the softmax and epilogue warps that O holds the step.
     __shared__ uint64_t bar_q, bar_qfree, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
-        bar_epi, bar_osc[2], bar_drain, bar_ready[2], bar_listfree, bar_infofree[2];
+        bar_epi, bar_osc[2], bar_drain, bar_ready[2], bar_listfree, bar_infofree[2], bar_creq[4][2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh, item_sh;
     __shared__ int n_ent_sh[3];
     __shared__ ItemInfo info_sh[2];    // per item parity: the work item and its step counts
     __shared__ float oscale_sh[2][128];  // per item parity and row: unit / l, for the epilogue
+    __shared__ float ofac_sh[2][128];    // per step parity and row: factor for O before the step's PV
 
     // warp index and everything derived from shared scalars are broadcast
     // from lane 0 so that the compiler treats them as warp-uniform
@@ -281,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
         mbar_init(&bar_s, 1);
         mbar_init(&bar_sfree, 4);  // one arrive per softmax warp
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar_p[s], 4);    // one arrive per softmax warp
+            mbar_init(&bar_p[s], 8);    // one arrive per softmax warp and per correction warp
+            for (int q = 0; q < 4; ++q) mbar_init(&bar_creq[q][s], 1);  // a softmax warp's O factors
             mbar_init(&bar_osc[s], 4);  // the softmax warps wrote an item's output scales
             mbar_init(&bar_ready[s], 1);      // the scheduler published an item
             mbar_init(&bar_infofree[s], 4);   // the epilogue warps are done with an item
@@ -687,6 +668,20 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                     // P buffer pb was last read by the PV of step g-2, which the MMA
                     // warp issued before S(g): the S commit awaited above covers it
                     uint8_t* pbuf = smem + L::p + pb * L::p_bytes;
+                    // Factor for O before this step's PV, handed to the correction
+                    // warp of this lane quarter as soon as it is known: the
+                    // running-max correction, times the change of units (Eq. 8) at
+                    // a phase switch, which applies to every row.  The factor buffer
+                    // of parity pb was read for step g-2 before that step's PV,
+                    // which the MMA warp issued before S(g).
+                    auto post_factor = [&](float c) {
+                        float f = c;
+                        if (j > 0 && j == n16e && n8e > 0) f *= f16_8;                   // 16-bit -> 8-bit units
+                        if (j > 0 && j == n16e + n8e) f *= n8e > 0 ? switch_f : f16_4;  // -> 4-bit units
+                        ofac_sh[pb][r] = j > 0 ? f : 1.0f;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar_creq[quarter][pb]);
+                    };
                     float corr = 1.0f;
                     if (active) {
                         // v = s * c (log2 units); the winning key gets v - m = 0
@@ -737,6 +732,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                         const float mn = fmaxf(m, rmx);
                         if (m != -INFINITY && mn > m) corr = ex2f(m - mn);
                         m = mn;
+                        post_factor(corr);
                         const float2 nm = make_float2(-mn, -mn);
                         const float2 rt = make_float2(mt.ratio, mt.ratio);
                         float2 acc0 = make_float2(0.0f, 0.0f), acc1 = acc0;
@@ -827,6 +823,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                         l = l * corr + (a2.x + a2.y);
                     } else {
                         // row not in this step: zero weights
+                        post_factor(1.0f);
                         if (T16 && ph == 2) {
 #pragma unroll
                             for (int ch = 0; ch < 8; ++ch)
@@ -845,44 +842,9 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                             *reinterpret_cast<uint32_t*>(sfp) = 0u;
                         }
                     }
-                    // factor for O before this step's PV: the running-max correction,
-                    // times the change of units (sigma8 -> sigma4) at the switch from
-                    // the 8-bit to the 4-bit phase, which applies to every row
-                    float f = corr;
-                    if (j > 0 && j == n16e && n8e > 0) f *= f16_8;  // 16-bit -> 8-bit units
-                    if (j > 0 && j == n16e + n8e) f *= n8e > 0 ? switch_f : f16_4;  // -> 4-bit units
-                    // O rescale (this thread's row), when the row max grew or the
-                    // units change; O must hold the PV of step g-1 first, which was
-                    // issued a whole step ago
-                    const bool need = (f != 1.0f) && j > 0;
-                    if (__any_sync(0xffffffffu, need)) {
-                        const uint32_t gp = g - 1;
-                        const bool w2 =
-                            mbar_wait(&bar_empty[gp % kStages], (gp / kStages) & 1, abort_v, p.status, p.wait_ns);
-                        if (!__all_sync(0xffffffffu, w2)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint64_t f2 = need ? pack2(f, f) : pack2(1.0f, 1.0f);
-#pragma unroll 1
-                        for (int c0 = 0; c0 < D; c0 += 64) {
-                            uint32_t o[64];
-                            tmem_ld32x2(lane_base + kColO + c0, o);
-#pragma unroll
-                            for (int c = 0; c < 64; c += 2) {
-                                const uint64_t x = mul2(pack2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), f2);
-                                o[c] = __float_as_uint(lo2(x));
-                                o[c + 1] = __float_as_uint(hi2(x));
-                            }
-                            tmem_st32x2(lane_base + kColO + c0, o);
-                        }
-                        tc_wait_st();
-                    }
                     // every thread makes its weight stores visible to the tensor
                     // core; after the warp barrier one lane publishes them
                     fence_proxy_async_smem();
-                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bar_p[pb]);
                 }
@@ -921,8 +883,51 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                 const bool qvalid = hf == 0 || has1;
                 const int a = qvalid && hf ? a1 : a0;
                 const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-                // the softmax warps' output scales of this item
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_osc[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns));
+                // ---- O correction, step by step: once the softmax warp of this
+                // quarter posted the step's factors, rows whose factor is not 1
+                // are rescaled in O (which must hold the PV of the previous step
+                // first), then this warp's arrive completes, with the softmax
+                // warps', the step's P barrier
+                bool cok = true;
+                for (int j = 0; j < n_ent; ++j) {
+                    const uint32_t g = gstep + j, pb = g & 1;
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(&bar_creq[quarter][pb], (g >> 1) & 1, abort_v, p.status, p.wait_ns))) {
+                        cok = false;
+                        break;
+                    }
+                    const float f = ofac_sh[pb][r];
+                    if (__any_sync(0xffffffffu, f != 1.0f)) {
+                        // a factor other than 1 only from the second step on
+                        const uint32_t gp = g - 1;
+                        const bool w2 =
+                            mbar_wait(&bar_empty[gp % kStages], (gp / kStages) & 1, abort_v, p.status, p.wait_ns);
+                        if (!__all_sync(0xffffffffu, w2)) {
+                            cok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t f2 = pack2(f, f);
+#pragma unroll 1
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(lane_base + kColO + c0, o);
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2) {
+                                const uint64_t x = mul2(pack2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), f2);
+                                o[c] = __float_as_uint(lo2(x));
+                                o[c + 1] = __float_as_uint(hi2(x));
+                            }
+                            tmem_st32(lane_base + kColO + c0, o);
+                        }
+                        tc_wait_st();
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar_p[pb]);
+                }
+                // ---- epilogue: the softmax warps' output scales of this item
+                bool ok = cok && __all_sync(0xffffffffu, mbar_wait(&bar_osc[k & 1], (k >> 1) & 1, abort_v, p.status, p.wait_ns));
                 float o_scale = 0.0f;
                 const bool have = n_ent > 0 && ok;
                 if (have) {
