@@ -43,6 +43,43 @@ __device__ __forceinline__ uint32_t kmajor_offset(int row, int chunk, int row_by
     return ((row >> 3) * (row_bytes >> 4) + chunk) * 128 + (row & 7) * 16;
 }
 
+// Four fp32 -> four e4m3 bytes in one word (first value in the low byte),
+// round to nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x4(float2 a, float2 b) {
+    uint32_t w;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return w;
+}
+// Eight fp32 -> eight e2m1 nibbles in one word (first value in the low
+// nibble), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+    return w;
+}
+// Largest |x| of the bf16 pairs in n words, per half: |x| of a finite bf16
+// orders like its 15 magnitude bits.
+template <int N>
+__device__ __forceinline__ uint32_t absmax_bf16x2(const uint32_t* w) {
+    uint32_t m = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 1; i + 1 < N; i += 2) m = __vimax3_u16x2(m, w[i] & 0x7FFF7FFFu, w[i + 1] & 0x7FFF7FFFu);
+    if constexpr (N % 2 == 0) m = __vmaxu2(m, w[N - 1] & 0x7FFF7FFFu);
+    return m;
+}
+
 template <int D>
 __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_kernel(PrepareArgs p) {
     constexpr int kThreads = threads_for<D>();
@@ -144,41 +181,26 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
     uint8_t* dst4 = (which == 0 ? p.q4 : (which == 1 ? p.k4 : p.v4)) + ba * (size_t)(32 * D);
     // FP8 e4m3 of 16 values: e4m3(RN(x * inv8)), 0 for a zero tile
     auto fp8x16 = [&](const float* x) -> uint4 {
+        if (zero) return make_uint4(0u, 0u, 0u, 0u);
+        const float2 s2 = make_float2(inv8, inv8);
         uint32_t w[4];
 #pragma unroll
-        const float2 s2 = make_float2(inv8, inv8);
-        for (int e = 0; e < 4; ++e) {
-            const float2 y0 = __fmul2_rn(make_float2(x[4 * e], x[4 * e + 1]), s2);
-            const float2 y1 = __fmul2_rn(make_float2(x[4 * e + 2], x[4 * e + 3]), s2);
-            const uint16_t lo = zero ? 0 : cvt_e4m3x2(y0.x, y0.y);
-            const uint16_t hi = zero ? 0 : cvt_e4m3x2(y1.x, y1.y);
-            w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
-        }
+        for (int e = 0; e < 4; ++e)
+            w[e] = e4m3x4(__fmul2_rn(make_float2(x[4 * e], x[4 * e + 1]), s2),
+                          __fmul2_rn(make_float2(x[4 * e + 2], x[4 * e + 3]), s2));
         return make_uint4(w[0], w[1], w[2], w[3]);
     };
-    // NVFP4 group of 16 values: scale byte sf = e4m3(RN(amax16 * 448/amax)),
-    // codes e2m1(RN(x * RN(1 / RN(value(sf) * g4)))) into 8 bytes
-    auto fp4x16 = [&](const float* x, uint8_t* sf_out) -> uint2 {
-        float a16 = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) a16 = max3f(a16, fabsf(x[e]), fabsf(x[e + 1]));
+    // NVFP4 group of 16 values with largest magnitude a16: scale byte
+    // sf = e4m3(RN(a16 * 448/amax)), codes e2m1(RN(x * RN(1 / RN(value(sf) * g4))))
+    // into 8 bytes
+    auto fp4x16 = [&](const float* x, float a16, uint8_t* sf_out) -> uint2 {
         const uint32_t sf = zero ? 0u : (uint32_t)(cvt_e4m3x2(__fmul_rn(a16, t4), 0.0f) & 0xFF);
         *sf_out = (uint8_t)sf;
         if (sf == 0) return make_uint2(0u, 0u);
         const float rcp = __frcp_rn(__fmul_rn(e4m3_to_f32((uint8_t)sf), g4));
         const float2 r2 = make_float2(rcp, rcp);
-        uint32_t w[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            uint32_t acc = 0;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 y = __fmul2_rn(make_float2(x[8 * h + 2 * e], x[8 * h + 2 * e + 1]), r2);
-                acc |= (uint32_t)cvt_e2m1x2(y.x, y.y) << (8 * e);
-            }
-            w[h] = acc;
-        }
-        return make_uint2(w[0], w[1]);
+        auto y = [&](int i) { return __fmul2_rn(make_float2(x[i], x[i + 1]), r2); };
+        return make_uint2(e2m1x8(y(0), y(2), y(4), y(6)), e2m1x8(y(8), y(10), y(12), y(14)));
     };
     auto bf_lo = [](uint32_t w) { return __uint_as_float(w << 16); };
     auto bf_hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
@@ -189,23 +211,31 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
         for (int it = tid; it < 64 * (D / 32); it += kThreads) {
             const int r = it & 63, k = it >> 6;
             float x[32];
-            uint4 raw[4];
+            uint32_t ww[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                raw[q] = *reinterpret_cast<const uint4*>(&tile[r * LD + 32 * k + 8 * q]);
-                const uint32_t ww[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[8 * q + 2 * e] = bf_lo(ww[e]);
-                    x[8 * q + 2 * e + 1] = bf_hi(ww[e]);
-                }
+                const uint4 raw = *reinterpret_cast<const uint4*>(&tile[r * LD + 32 * k + 8 * q]);
+                ww[4 * q] = raw.x;
+                ww[4 * q + 1] = raw.y;
+                ww[4 * q + 2] = raw.z;
+                ww[4 * q + 3] = raw.w;
             }
+            // largest magnitude of each 16-channel group (8 words each)
+            const uint32_t m0 = absmax_bf16x2<8>(ww), m1 = absmax_bf16x2<8>(ww + 8);
+            const float a0 = __uint_as_float(max(m0 & 0xFFFFu, m0 >> 16) << 16);
+            const float a1 = __uint_as_float(max(m1 & 0xFFFFu, m1 >> 16) << 16);
             if (p.q16) {
                 // bf16 tile of the 16-bit path: the input values as they are (2D-byte rows)
                 uint8_t* dst16 = (which == 0 ? p.q16 : p.k16) + ba * (size_t)(128 * D);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(dst16 + kmajor_offset(r, 4 * k + q, 2 * D)) = raw[q];
+                    *reinterpret_cast<uint4*>(dst16 + kmajor_offset(r, 4 * k + q, 2 * D)) =
+                        make_uint4(ww[4 * q], ww[4 * q + 1], ww[4 * q + 2], ww[4 * q + 3]);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                x[2 * e] = bf_lo(ww[e]);
+                x[2 * e + 1] = bf_hi(ww[e]);
             }
             if (p.q8i) {
                 int8_t* dsti = (which == 0 ? p.q8i : p.k8i) + ba * (size_t)(64 * D);
@@ -227,7 +257,7 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
             *reinterpret_cast<uint4*>(dst8 + kmajor_offset(r, 2 * k, D)) = fp8x16(x);
             *reinterpret_cast<uint4*>(dst8 + kmajor_offset(r, 2 * k + 1, D)) = fp8x16(x + 16);
             uint8_t sf0, sf1;
-            const uint2 c0 = fp4x16(x, &sf0), c1 = fp4x16(x + 16, &sf1);
+            const uint2 c0 = fp4x16(x, a0, &sf0), c1 = fp4x16(x + 16, a1, &sf1);
             *reinterpret_cast<uint4*>(dst4 + kmajor_offset(r, k, D / 2)) = make_uint4(c0.x, c0.y, c1.x, c1.y);
 #pragma unroll
             for (int gi = 0; gi < 2; ++gi) {
@@ -242,24 +272,18 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
         // read gives both channels of a slot, a warp reads 128 contiguous bytes
         for (int it = tid; it < (D / 2) * 4; it += kThreads) {
             const int c = it % (D / 2), k = it / (D / 2);
-            float x0[16], x1[16];
-            uint32_t b16[2][8];  // bf16 pairs of V^T rows 2c and 2c+1 (slots 16k..16k+15)
+            uint32_t w[16];  // slot sl of the group: channel 2c in the low half, 2c+1 in the high half
 #pragma unroll
-            for (int sl = 0; sl < 16; ++sl) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(&tile[(16 * k + sl) * LD + 2 * c]);
-                x0[sl] = bf_lo(w);
-                x1[sl] = bf_hi(w);
-                if (sl & 1) {
-                    b16[0][sl >> 1] |= (w & 0xFFFFu) << 16;
-                    b16[1][sl >> 1] |= w & 0xFFFF0000u;
-                } else {
-                    b16[0][sl >> 1] = w & 0xFFFFu;
-                    b16[1][sl >> 1] = w >> 16;
-                }
-            }
+            for (int sl = 0; sl < 16; ++sl) w[sl] = *reinterpret_cast<const uint32_t*>(&tile[(16 * k + sl) * LD + 2 * c]);
             if (p.v16) {
                 // bf16 V^T of the 16-bit path: rows 2c and 2c+1, 32 bytes each (128-byte rows)
                 uint8_t* dst16 = p.v16 + ba * (size_t)(128 * D);
+                uint32_t b16[2][8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    b16[0][i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x5410);
+                    b16[1][i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x7632);
+                }
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
@@ -267,13 +291,18 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
                         *reinterpret_cast<uint4*>(dst16 + kmajor_offset(2 * c + hh, 2 * k + q, 128)) =
                             make_uint4(b16[hh][4 * q], b16[hh][4 * q + 1], b16[hh][4 * q + 2], b16[hh][4 * q + 3]);
             }
+            // largest magnitude of the group in each channel
+            const uint32_t m2 = absmax_bf16x2<16>(w);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int row = 2 * c + h;
-                const float* x = h ? x1 : x0;
+                float x[16];
+#pragma unroll
+                for (int sl = 0; sl < 16; ++sl) x[sl] = h ? bf_hi(w[sl]) : bf_lo(w[sl]);
                 *reinterpret_cast<uint4*>(dst8 + kmajor_offset(row, k, 64)) = fp8x16(x);
                 uint8_t sf;
-                const uint2 c4 = fp4x16(x, &sf);
+                const float a16 = __uint_as_float((h ? m2 >> 16 : m2 & 0xFFFFu) << 16);
+                const uint2 c4 = fp4x16(x, a16, &sf);
                 *reinterpret_cast<uint2*>(dst4 + kmajor_offset(row, k >> 1, 32) + 8 * (k & 1)) = c4;
                 sf_atom[16 * (row & 31) + 4 * (row >> 5) + k] = sf;
             }
