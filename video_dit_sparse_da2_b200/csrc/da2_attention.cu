@@ -70,7 +70,7 @@ constexpr int kMmaWarp = 8, kLoadWarp = 9;
 // Registers per thread: every thread starts with kRegLaunch (two CTAs of 384
 // threads share the 64K registers of an SM); the warpgroups then move to
 // their own budgets, whose sum is the CTA's allocation.
-constexpr uint32_t kRegLaunch = 80, kRegSoftmax = 160, kRegCorr = 48, kRegAux = 32;
+constexpr uint32_t kRegLaunch = 80, kRegSoftmax = 152, kRegCorr = 48, kRegAux = 40;
 static_assert((kRegSoftmax + kRegCorr + kRegAux) * 128 == kRegLaunch * kThreads,
               "the warpgroup register budgets must add up to the launch allocation");
 static_assert(2 * kRegLaunch * kThreads <= 65536, "two CTAs per SM");
