@@ -57,6 +57,9 @@ struct PlanArgs {
     SelectTarget* sel;       // [BH][3] (scratch): 16-bit, 8-bit, kept cuts
     unsigned int* hist;      // [BH][3][4096] (scratch)
     unsigned int* done_count;  // [BH] finished histogram CTAs of the current pass (scratch)
+    int* cand_n;              // [BH] keys in the head's selection candidate list (scratch; the
+                              //   list itself sits in the head's Lmax rows, dead after the softmax)
+    int* cand_state;          // [BH] 0 no list, 1 list collected (later passes read it)
     uint8_t* prec;           // [BH][R][R]
     int32_t* cnt;            // [3][BH][R]: 8-bit, 4-bit, 16-bit counts
     long long* off;          // [BH][R+1] list offsets (positions in kidx)

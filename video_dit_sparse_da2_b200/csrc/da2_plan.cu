@@ -251,6 +251,16 @@ struct Key {
 };
 
 constexpr int kTargets = 3;  // selection targets per head (16-bit, 8-bit, kept cuts)
+// Keys a head's candidate list holds at most: the first pass in which the open
+// targets' prefixes match at most this many keys in all collects them, and the
+// later passes read the list instead of the whole draft map.  The list (A bits,
+// then ~pair index) sits in the head's rows of the max-branch logits, which the
+// softmax kernel has consumed: R^2 doubles hold min(kSelectCand, 2 R^2 / 3) keys.
+constexpr int kSelectCand = 16384;
+__host__ __device__ inline int select_cand_cap(int R) {
+    const long long c = 2ll * R * R / 3;
+    return c < kSelectCand ? (int)c : kSelectCand;
+}
 
 __device__ __forceinline__ void top_mask(int nbits, unsigned long long* mh, unsigned int* ml) {
     *mh = nbits <= 0 ? 0ull : (nbits >= 64 ? ~0ull : (~0ull << (64 - nbits)));
@@ -288,6 +298,8 @@ __global__ void select_init_kernel(PlanArgs p, long long C16, long long C8, long
         s.key_lo = 0u;
         p.sel[bh * kTargets + t] = s;
     }
+    p.cand_n[bh] = 0;
+    p.cand_state[bh] = 0;
 }
 
 constexpr int kHistThreads = 1024;
@@ -398,14 +410,27 @@ __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, i
     const size_t RR = (size_t)p.R * p.R;
     const size_t begin = (size_t)blockIdx.x * chunk;
     const double* Ah = p.A + (size_t)bh * RR;
-    auto count = [&](size_t i, double a) {
-        Key k;
-        k.hi = (unsigned long long)__double_as_longlong(a);
-        k.lo = 0xFFFFFFFFu - (unsigned)i;
+    // candidate list: read it once collected; collect it in the first pass in
+    // which the open targets match at most kSelectCand keys together (a key
+    // matching any open prefix is kept: the prefixes only grow from here)
+    long long live = 0;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+        if (!s[t].done) live += s[t].unique ? 1 : s[t].matches;
+    const int cap = select_cand_cap(p.R);
+    const int cstate = p.cand_state[bh];
+    const bool from_list = cstate == 1, collect = cstate == 0 && live <= cap;
+    unsigned long long* ch = reinterpret_cast<unsigned long long*>(p.Lmax + (size_t)bh * RR);
+    unsigned* cl = reinterpret_cast<unsigned*>(ch + cap);
+    // histogram (or record) key k for every open target whose prefix it
+    // matches; true when it matches one
+    auto count_key = [&](Key k) -> bool {
+        bool any = false;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             if (s[t].done) continue;
             if (((k.hi ^ s[t].p_hi) & mh[t]) || ((k.lo ^ s[t].p_lo) & ml[t])) continue;
+            any = true;
             if (s[t].unique) {
                 p.sel[bh * kTargets + t0 + t].key_hi = k.hi;
                 p.sel[bh * kTargets + t0 + t].key_lo = k.lo;
@@ -416,20 +441,48 @@ __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, i
                 atomicAdd(&gh[t * 4096 + digit_at(k, pos[t], w[t])], 1u);
             }
         }
+        return any;
     };
-    // chunk / kHistThreads keys per thread (a multiple of 4), four loads in flight
-#pragma unroll 1
-    for (int k0 = 0; k0 < chunk / kHistThreads; k0 += 4) {
-        double a[4];
-        size_t idx[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            idx[u] = begin + (size_t)(k0 + u) * kHistThreads + tid;
-            a[u] = idx[u] < RR ? __ldcs(Ah + idx[u]) : 0.0;
+    auto count = [&](size_t i, double a) {
+        Key k;
+        k.hi = (unsigned long long)__double_as_longlong(a);
+        k.lo = 0xFFFFFFFFu - (unsigned)i;
+        if (count_key(k) && collect) {
+            // at most `live` keys match an open prefix, so the list cannot overflow
+            const int slot = atomicAdd(&p.cand_n[bh], 1);
+            if (slot < cap) {
+                ch[slot] = k.hi;
+                cl[slot] = k.lo;
+            }
         }
+    };
+    if (from_list) {
+        // the keys still in play were collected by an earlier pass: the first
+        // CTA of the head goes through them, the others only report
+        if (blockIdx.x == 0) {
+            const int n = min(__ldcg(&p.cand_n[bh]), cap);
+            for (int i = tid; i < n; i += kHistThreads) {
+                Key k;
+                k.hi = __ldcg(&ch[i]);
+                k.lo = __ldcg(&cl[i]);
+                count_key(k);
+            }
+        }
+    } else {
+        // chunk / kHistThreads keys per thread (a multiple of 4), four loads in flight
+#pragma unroll 1
+        for (int k0 = 0; k0 < chunk / kHistThreads; k0 += 4) {
+            double a[4];
+            size_t idx[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (idx[u] < RR) count(idx[u], a[u]);
+            for (int u = 0; u < 4; ++u) {
+                idx[u] = begin + (size_t)(k0 + u) * kHistThreads + tid;
+                a[u] = idx[u] < RR ? __ldcs(Ah + idx[u]) : 0.0;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (idx[u] < RR) count(idx[u], a[u]);
+        }
     }
     if (any_smem) {
         __syncthreads();
@@ -446,7 +499,10 @@ __global__ void __launch_bounds__(kHistThreads) select_hist_kernel(PlanArgs p, i
     if (!is_last) return;
     __threadfence();
     if (tid < 32 * NT) select_scan_warp(p, bh, t0 + (tid >> 5), tid & 31);
-    if (tid == 0) p.done_count[bh] = 0u;
+    if (tid == 0) {
+        p.done_count[bh] = 0u;
+        if (collect) p.cand_state[bh] = 1;  // every CTA of the head has appended its keys
+    }
 }
 
 // ---------------------------------------------------------------- classify
@@ -691,6 +747,8 @@ size_t plan_scratch_bytes(int BH, int R, int d) {
     b = (b + 255) & ~(size_t)255;
     b += (size_t)BH * sizeof(unsigned);
     b = (b + 255) & ~(size_t)255;
+    b += (size_t)2 * BH * sizeof(int);  // candidate list counts and states
+    b = (b + 255) & ~(size_t)255;
     b += mx_scratch_bytes(BH, R, d);  // split descriptors of the exact max-pool branch
     return b;
 }
@@ -710,6 +768,11 @@ void plan_carve_scratch(PlanArgs* p, void* scratch) {
     off = (off + 255) & ~(size_t)255;
     p->done_count = reinterpret_cast<unsigned*>(c + off);
     off += (size_t)p->BH * sizeof(unsigned);
+    off = (off + 255) & ~(size_t)255;
+    p->cand_n = reinterpret_cast<int*>(c + off);
+    off += (size_t)p->BH * sizeof(int);
+    p->cand_state = reinterpret_cast<int*>(c + off);
+    off += (size_t)p->BH * sizeof(int);
     off = (off + 255) & ~(size_t)255;
     mx_carve(p, c + off);
 }
