@@ -61,9 +61,9 @@ namespace {
 
 constexpr int kStages = 3;
 // Roles: softmax warps 0-3 (one thread per tile row, all 64 key columns of a
-// step), epilogue warps 4-7 (one thread per tile row), MMA warp 8, loader
-// warp 9, scheduler warps 10-11 (the register budgets are set per warpgroup
-// of four warps).
+// step), correction and epilogue warps 4-7 (one thread per tile row), MMA
+// warp 8, loader warp 9, scheduler warps 10-11 (the register budgets are set
+// per warpgroup of four warps).
 constexpr int kSoftmaxThreads = 128;
 constexpr int kThreads = 384;
 constexpr int kMmaWarp = 8, kLoadWarp = 9;
@@ -156,32 +156,6 @@ __device__ __forceinline__ void tmem_ld64x2_rec(uint32_t taddr, uint32_t raddr, 
         : "memory");
 }
 
-// Four fp32 -> four e4m3 bytes in one word (first value in the low byte).
-__device__ __forceinline__ uint32_t pack_e4m3x4(float2 a, float2 b) {
-    uint32_t w;
-    asm("{\n\t.reg .b16 lo, hi;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
-        "mov.b32 %0, {lo, hi};\n\t}"
-        : "=r"(w)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return w;
-}
-
-// Eight fp32 -> eight e2m1 nibbles in one word (first value in the low nibble).
-__device__ __forceinline__ uint32_t pack_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
-    uint32_t w;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(w)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
-    return w;
-}
-
 // Max of the 16 consecutive values v[b..b+7] (pairs).
 template <int NP>
 __device__ __forceinline__ float groupmax16_raw(const float2 (&v)[NP], int b) {
@@ -228,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
     extern __shared__ __align__(1024) uint8_t smem[];
     // bar_empty[st] completes when the PV of a step in stage st has finished:
     // it frees the stage for the loader, frees that step's P buffer two steps
-    // later, and tells the softmax and epilogue warps that O holds the step.
+    // later, and tells the correction and epilogue warps that O holds the step.
     __shared__ uint64_t bar_q, bar_qfree, bar_sfq, bar_full[kStages], bar_empty[kStages], bar_s, bar_sfree, bar_p[2],
         bar_epi, bar_osc[2], bar_drain, bar_ready[2], bar_listfree, bar_infofree[2], bar_creq[4][2];
     __shared__ uint32_t tmem_base_sh;
@@ -443,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, T16 ? 1 : 2) attention_kernel(AttnAr
                                  tmem + kColSfp + 4 * pb, tmem + kColSfv + 4 * pb, i > 0 ? 1u : 0u);
                     }
                     // frees the stage and (two steps later) the P buffer, and tells
-                    // the softmax and epilogue warps that O holds step g
+                    // the correction and epilogue warps that O holds step g
                     tc_commit_w(&bar_empty[st]);
                     return true;
                 };

@@ -257,14 +257,34 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
         : "f"(hi), "f"(lo));
     return r;
 }
-// Two fp32 values -> one byte of two e2m1 codes; `lo` in the low nibble.
-__device__ __forceinline__ uint8_t cvt_e2m1x2(float lo, float hi) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-        : "=r"(r)
-        : "f"(hi), "f"(lo));
-    return (uint8_t)r;
+// Four fp32 -> four e4m3 bytes in one word (first value in the low byte),
+// round to nearest even, saturating.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float2 a, float2 b) {
+    uint32_t w;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return w;
 }
+
+// Eight fp32 -> eight e2m1 nibbles in one word (first value in the low
+// nibble), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t pack_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+    return w;
+}
+
 // Exact value of an e4m3 byte (through the half-precision converter).
 __device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
     uint32_t h2;

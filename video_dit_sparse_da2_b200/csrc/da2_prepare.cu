@@ -43,32 +43,6 @@ __device__ __forceinline__ uint32_t kmajor_offset(int row, int chunk, int row_by
     return ((row >> 3) * (row_bytes >> 4) + chunk) * 128 + (row & 7) * 16;
 }
 
-// Four fp32 -> four e4m3 bytes in one word (first value in the low byte),
-// round to nearest even, saturating.
-__device__ __forceinline__ uint32_t e4m3x4(float2 a, float2 b) {
-    uint32_t w;
-    asm("{\n\t.reg .b16 lo, hi;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
-        "mov.b32 %0, {lo, hi};\n\t}"
-        : "=r"(w)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return w;
-}
-// Eight fp32 -> eight e2m1 nibbles in one word (first value in the low
-// nibble), round to nearest even, saturating.
-__device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
-    uint32_t w;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(w)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
-    return w;
-}
 // Largest |x| of the bf16 pairs in n words, per half: |x| of a finite bf16
 // orders like its 15 magnitude bits.
 template <int N>
@@ -186,8 +160,8 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            w[e] = e4m3x4(__fmul2_rn(make_float2(x[4 * e], x[4 * e + 1]), s2),
-                          __fmul2_rn(make_float2(x[4 * e + 2], x[4 * e + 3]), s2));
+            w[e] = pack_e4m3x4(__fmul2_rn(make_float2(x[4 * e], x[4 * e + 1]), s2),
+                               __fmul2_rn(make_float2(x[4 * e + 2], x[4 * e + 3]), s2));
         return make_uint4(w[0], w[1], w[2], w[3]);
     };
     // NVFP4 group of 16 values with largest magnitude a16: scale byte
@@ -200,7 +174,7 @@ __global__ void __launch_bounds__(threads_for<D>(), min_ctas_for<D>()) prepare_k
         const float rcp = __frcp_rn(__fmul_rn(e4m3_to_f32((uint8_t)sf), g4));
         const float2 r2 = make_float2(rcp, rcp);
         auto y = [&](int i) { return __fmul2_rn(make_float2(x[i], x[i + 1]), r2); };
-        return make_uint2(e2m1x8(y(0), y(2), y(4), y(6)), e2m1x8(y(8), y(10), y(12), y(14)));
+        return make_uint2(pack_e2m1x8(y(0), y(2), y(4), y(6)), pack_e2m1x8(y(8), y(10), y(12), y(14)));
     };
     auto bf_lo = [](uint32_t w) { return __uint_as_float(w << 16); };
     auto bf_hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
