@@ -33,7 +33,7 @@ METRIC = "ms/call and dense-equiv TFLOPS at 1 B200; % of mixed FP8/FP4 tensor ro
 # the attention sources whose hash is given; any other source or workload
 # reports null.  Filled in only from a capture of the current kernel.
 ATTN_TRAFFIC: dict = {
-    "hunyuanvideo-720p": {"bytes": 999.45e6 + 695.76e6, "sources_sha256_16": "a910aa82fbef154d"},
+    "hunyuanvideo-720p": {"bytes": 1.00e9 + 695.82e6, "sources_sha256_16": "d52ed58f63147302"},
 }
 _ATTN_SOURCES = ("video_dit_sparse_da2_b200/csrc/da2_attention.cu", "video_dit_sparse_da2_b200/csrc/da2_common.cuh")
 
